@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the Shampoo optimizer step (statistics + inverse roots +
+grafted apply) on B200, through the library's C-ABI.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                  [--config transformer_layer_b512]
+
+A step is update_stats, compute_roots on every root_interval-th step
+(counted from the first timed step, so K = root_interval times the root
+step exactly once per interval) and apply, on one fixed seeded gradient set
+per step.  Inputs are resident in HBM before timing; each step is timed with
+CUDA events on the optimizer's stream and L2 is flushed (a 256 MiB write)
+between steps, outside the events.  With N > 1 (torchrun) every rank runs its
+own copy of the parameter set: the blocks are independent, so there is no
+data-path collective (weak scaling); the job time is the max over ranks.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from shampoo_second_order_b200 import workloads as wl  # noqa: E402
+
+METRIC = "Shampoo optimizer step ms and TFLOP/s (stats+roots+apply) vs B200 peak, 1 GPU"
+UNIT = "TFLOP/s"
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
+# ncu capture of the named kernel; None until measured for the current kernel.
+TRAFFIC_PER_LAUNCH = {}
+
+
+# ---------------------------------------------------------------------------
+# Work model: algorithmic flops and bytes of the workload
+# ---------------------------------------------------------------------------
+def blocks_of(cfg):
+    b = cfg["block_size"]
+    blks, segs = [], []
+    for s in cfg["shapes"]:
+        if len(s) == 2:
+            for r0 in range(0, s[0], b):
+                for c0 in range(0, s[1], b):
+                    blks.append((min(b, s[0] - r0), min(b, s[1] - c0)))
+        else:
+            for s0 in range(0, s[0], b):
+                segs.append(min(b, s[0] - s0))
+    return blks, segs
+
+
+def matrix_sizes(cfg):
+    """(valid side, products per Newton step) per statistic, library order."""
+    blks, segs = blocks_of(cfg)
+    out = []
+    for m, n in blks:
+        out += [(m, 4 if cfg["p"] == 4 else 3), (n, 4 if cfg["p"] == 4 else 3)]
+    out += [(ln, 3 if cfg["p"] == 4 else 3) for ln in segs]   # p/2 = 2: X T, T T, T^2 M
+    return out
+
+
+def stats_flops(cfg):
+    """SYRK triangles: m(m+1) n for L and n(n+1) m for R; len(len+1) per segment."""
+    blks, segs = blocks_of(cfg)
+    return sum(m * (m + 1) * n + n * (n + 1) * m for m, n in blks) + sum(l * (l + 1) for l in segs)
+
+
+def apply_flops(cfg):
+    """Two chained GEMMs per block, 2mn(m+n); a matvec 2 len^2 per segment."""
+    blks, segs = blocks_of(cfg)
+    return sum(2 * m * n * (m + n) for m, n in blks) + sum(2 * l * l for l in segs)
+
+
+def newton_flops(cfg, iters, per_kernel=False):
+    """Symmetric products: n^2 (n+1) flops each (the upper triangle), times
+    products per step, times the iterations each matrix ran."""
+    sizes = matrix_sizes(cfg)
+    a = b = c = 0
+    for (n, prods), k in zip(sizes, iters):
+        k = k if k >= 0 else -1 - k
+        f = n * n * (n + 1)
+        a += 2 * k * f
+        b += (k * f) if prods == 4 else 0
+        c += k * f
+    return (a, b, c) if per_kernel else a + b + c
+
+
+def numel(cfg):
+    return wl.count_params(cfg["shapes"])
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if uuid:
+            cmd += ["-i", uuid]
+        try:
+            self.p = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def fp64_peak_tflops(torch, dev):
+    """cuBLAS DGEMM throughput (torch.matmul, float64, 4096^3, best of 5)."""
+    n = 4096
+    a = torch.randn(n, n, dtype=torch.float64, device=dev)
+    b = torch.randn(n, n, dtype=torch.float64, device=dev)
+    torch.matmul(a, b)
+    best = 1e9
+    for _ in range(5):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        torch.matmul(a, b)
+        e.record()
+        e.synchronize()
+        best = min(best, s.elapsed_time(e))
+    del a, b
+    return 2 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak):
+    """Achieved vs peak for the kernel with the largest share of device time."""
+    names = {k: v for k, v in prof.items() if v[1] > 0}
+    if not names:
+        return None, None
+    top = max(names, key=lambda k: names[k][1])
+    launches, ms = names[top]
+    hbm = peaks["hbm_gbs"]
+    blks, segs = blocks_of(cfg)
+    el = numel(cfg)
+    gbytes = 2 if cfg["grad_dtype"] == "bf16" else 4
+    work = None
+    if top.startswith("newton_step"):
+        a, b, c = newton_flops(cfg, iters_sum, per_kernel=True)
+        fl = {"newton_step_a": a, "newton_step_b": b, "newton_step_c": c}[top]
+        work = ("tensor", fl / 1e12 / (ms * 1e-3), fp64_peak, "TFLOP/s", fl / max(launches, 1))
+    elif top == "stats_blocks":
+        fl = (stats_flops(cfg) - sum(l * (l + 1) for l in segs)) * steps
+        work = ("alu", fl / 1e12 / (ms * 1e-3), 74.4, "TFLOP/s", fl / max(launches, 1))
+    elif top in ("precond_y", "precond_p"):
+        fl = sum(2 * m * n * (n if top == "precond_y" else m) for m, n in blks) * steps
+        work = ("alu", fl / 1e12 / (ms * 1e-3), 74.4, "TFLOP/s", fl / max(launches, 1))
+    elif top == "update":
+        by = el * (4 + 8 + (8 if cfg["momentum"] else 0)) * steps
+        work = ("hbm", by / 1e9 / (ms * 1e-3), hbm, "GB/s", by / max(launches, 1))
+    elif top in ("dnorm", "diag_update", "check_finite"):
+        per = {"dnorm": gbytes + 4, "diag_update": gbytes + 8, "check_finite": gbytes}[top]
+        by = el * per * steps
+        work = ("hbm", by / 1e9 / (ms * 1e-3), hbm, "GB/s", by / max(launches, 1))
+    if work is None:
+        return top, None
+    bound, ach, peak, unit, per_launch = work
+    tr = TRAFFIC_PER_LAUNCH.get(top)
+    return top, {"kernel": top, "bound": bound, "achieved": round(ach, 3), "peak": round(peak, 2),
+                 "unit": unit, "frac": round(ach / peak, 4), "traffic": tr,
+                 "algorithmic_per_launch": per_launch, "launches": launches,
+                 "avg_launch_ms": round(ms / launches, 5),
+                 "peak_source": "cuBLAS DGEMM measured in this run" if bound == "tensor" else
+                 ("MEASURED_PEAKS.json hbm_gbs" if bound == "hbm" else
+                  "fp32 FMA units: 148 SMs x 128 lanes x 2 flop x 1.965 GHz")}
+
+
+# ---------------------------------------------------------------------------
+# CPU legs (oracle): the baseline line and the reference arm
+# ---------------------------------------------------------------------------
+def oracle_sample(cfg, n_steps):
+    """Time the fp64 oracle on the full workload: n_steps of stats + apply and
+    one root step; returns (seconds per step amortised over the root
+    interval, description)."""
+    from oracle import ShampooOracle
+    o = ShampooOracle(cfg["shapes"], cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"],
+                      cfg["graft"], cfg["momentum"])
+    W = [w.astype(np.float64) for w in wl.make_params(cfg["shapes"], cfg["seed"])]
+    g = wl.make_grads(cfg["shapes"], cfg["seed"], 0, cfg["grad_std"], cfg["grad_dtype"])
+    o.update_stats(g)
+    t0 = time.perf_counter()
+    o.compute_roots()
+    t_root = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    for t in range(n_steps):
+        o.update_stats(g)
+        W = o.apply(W, g, cfg["lr"])
+    t_sa = (time.perf_counter() - t0) / n_steps
+    return t_sa + t_root / cfg["root_interval"], t_root, t_sa
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def reference_arm(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    sizes = matrix_sizes(cfg)
+    from oracle import ShampooOracle
+    o = ShampooOracle(cfg["shapes"], cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"],
+                      cfg["graft"], cfg["momentum"])
+    W = [w.astype(np.float64) for w in wl.make_params(cfg["shapes"], cfg["seed"])]
+    grads = [wl.make_grads(cfg["shapes"], cfg["seed"], t, cfg["grad_std"], cfg["grad_dtype"])
+             for t in range(2)]
+    for t in range(args.warmup):
+        W = o.step(W, grads[t % 2], cfg["lr"], t == 0)
+    t0 = time.perf_counter()
+    n_root = 0
+    for j in range(args.steps):
+        r = j % cfg["root_interval"] == 0
+        n_root += r
+        W = o.step(W, grads[j % 2], cfg["lr"], r)
+    el = time.perf_counter() - t0
+    # The flops credited are the CUDA arm's: stats + apply per step and, per
+    # root step, the Newton products at the iteration count the CPU coupled
+    # Newton needs, here the mean over the first four statistics.
+    from oracle import coupled_newton_inverse_root
+    ks = [coupled_newton_inverse_root(A, cfg["eps"], p)[1] for A, p in o.matrices()[:4]]
+    k = int(round(sum(ks) / len(ks)))
+    fl = args.steps * (stats_flops(cfg) + apply_flops(cfg)) + n_root * newton_flops(cfg, [k] * len(sizes))
+    val = fl / el / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.config, "params": numel(cfg),
+                                            "block_size": cfg["block_size"]},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} full oracle steps ({n_root} with roots by eigh)"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--config", default="transformer_layer_b512", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    cfg = wl.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        return reference_arm(args, cfg, rank, world)
+
+    # CPU baseline first (rank 0, N = 1 only), before any GPU work
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        t_step, t_root, t_sa = oracle_sample(cfg, 2)
+        cpu = {"t_step_s": t_step, "t_root_s": t_root, "t_stats_apply_s": t_sa}
+
+    import torch
+    import torch.distributed as dist
+    from shampoo_second_order_b200 import Shampoo
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    stream = torch.cuda.Stream(device=dev)
+    peaks, peak_src = measured_peaks()
+    with torch.cuda.stream(stream):
+        fp64_peak = fp64_peak_tflops(torch, dev)
+    stream.synchronize()
+
+    shapes = cfg["shapes"]
+    gdt = torch.bfloat16 if cfg["grad_dtype"] == "bf16" else torch.float32
+    W0 = wl.make_params(shapes, cfg["seed"] + 17 * rank)
+    NG = 4
+    host_grads = [wl.make_grads(shapes, cfg["seed"] + 17 * rank, t, cfg["grad_std"], cfg["grad_dtype"])
+                  for t in range(NG)]
+    with torch.cuda.stream(stream):
+        W = [torch.from_numpy(w).to(dev) for w in W0]
+        G = [[torch.from_numpy(g).to(dev).to(gdt) for g in gs] for gs in host_grads]
+        flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    stream.synchronize()
+
+    opt = Shampoo(shapes, cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"], cfg["graft"],
+                  cfg["momentum"], cfg["grad_dtype"], stream=stream)
+    lr = cfg["lr"]
+    interval = cfg["root_interval"]
+
+    def step(gs, roots):
+        opt.update_stats(gs)
+        if roots:
+            opt.compute_roots()
+        opt.apply(W, gs, lr)
+
+    for t in range(args.warmup):
+        step(G[t % NG], t == 0)
+    stream.synchronize()
+
+    # ---- timed region: device-resident inputs ----
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    opt.profile_enable(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    iters_sum = [0] * opt.num_matrices()
+    n_root = 0
+    with torch.cuda.stream(stream):
+        for j in range(args.steps):
+            flush.zero_()
+            roots = j % interval == 0
+            ev[j][0].record(stream)
+            step(G[j % NG], roots)
+            ev[j][1].record(stream)
+            if roots:
+                n_root += 1
+                its = opt.root_iterations()
+                iters_sum = [a + (b if b >= 0 else -1 - b) for a, b in zip(iters_sum, its)]
+    stream.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    prof = opt.profile_read()
+    opt.profile_enable(False)
+    total_ms = sum(s.elapsed_time(e) for s, e in ev)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    launches = sum(v[0] for v in prof.values())
+
+    flops_rank = args.steps * (stats_flops(cfg) + apply_flops(cfg)) + newton_flops(cfg, iters_sum)
+    value = world * flops_rank / (total_ms * 1e-3) / 1e12
+
+    # ---- e2e: host buffers through the public API ----
+    e2e = None
+    if not args.no_e2e:
+        pin_g = [[torch.from_numpy(g).to(gdt).pin_memory() for g in gs] for gs in host_grads]
+        pin_w = [torch.empty(w.shape, dtype=torch.float32).pin_memory() for w in W0]
+        dG = [torch.empty_like(g) for g in G[0]]
+        h2d = sum(g.numel() * g.element_size() for g in pin_g[0])
+        d2h = sum(w.numel() * 4 for w in pin_w)
+        eve = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        with torch.cuda.stream(stream):
+            for j in range(args.steps):
+                flush.zero_()
+                eve[j][0].record(stream)
+                for d, h in zip(dG, pin_g[j % NG]):
+                    d.copy_(h, non_blocking=True)
+                step(dG, j % interval == 0)
+                for h, d in zip(pin_w, W):
+                    h.copy_(d, non_blocking=True)
+                eve[j][1].record(stream)
+        stream.synchronize()
+        e2e_ms = sum(s.elapsed_time(e) for s, e in eve)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * flops_rank / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms / args.steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak)
+
+    if rank == 0:
+        phase = {}
+        for k, (n, ms) in sorted(prof.items(), key=lambda kv: -kv[1][1]):
+            phase[k] = {"launches": n, "ms": round(ms, 4), "share": round(ms / max(total_ms, 1e-9), 4)}
+        cpu_line = None
+        if cpu is not None:
+            fl_amort = stats_flops(cfg) + apply_flops(cfg) + newton_flops(cfg, iters_sum) / max(args.steps, 1)
+            cpu_line = {"value": fl_amort / cpu["t_step_s"] / 1e12, "unit": UNIT, "cores": blas_threads(),
+                        "kind": "oracle",
+                        "sample": ("fp64 numpy oracle on the full workload: 2 steps of stats+apply and 1 "
+                                   "root step (eigh), amortised over the root interval"),
+                        "ms_per_step": cpu["t_step_s"] * 1e3}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
+            "config": {"workload": args.config, "params": numel(cfg), "block_size": cfg["block_size"],
+                       "grad_dtype": cfg["grad_dtype"], "root_interval": interval,
+                       "root_steps_timed": n_root, "l2": "flushed between steps (256 MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof, "cpu_baseline": cpu_line, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk, "kernels": phase, "fp64_gemm_peak_tflops": round(fp64_peak, 2),
+            "peaks_source": peak_src,
+            "flops_per_step": {"stats": stats_flops(cfg), "apply": apply_flops(cfg),
+                               "roots_per_root_step": newton_flops(cfg, iters_sum) / max(n_root, 1)},
+        }
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

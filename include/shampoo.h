@@ -1,0 +1,242 @@
+/*
+ * shampoo.h -- C-ABI of the B200 (sm_100a) Shampoo optimizer step.
+ *
+ * Shampoo preconditions each 2-D weight W (m x n) with two small matrices,
+ * L (rows) and R (columns), whose Kronecker product stands in for the full-
+ * matrix-Adagrad preconditioner ("Scalable Second Order Optimization for Deep
+ * Learning", Anil et al.; podcast transcript, segments 6-8).  One optimizer
+ * step is three pieces of extra work (same transcript, segment 10):
+ *
+ *   shampoo_update_stats   L <- beta2 L + G G^T,  R <- beta2 R + G^T G
+ *   shampoo_compute_roots  L^{-1/p}, R^{-1/p} by coupled Newton in float64
+ *                          (segment 12), only every so many steps (segment 14)
+ *   shampoo_apply          P = L^{-1/p} G R^{-1/p}, grafted to the norm of the
+ *                          diagonal-Adagrad step, momentum, weight update
+ *
+ * Large weights are split into <= b x b blocks, each with its own L and R
+ * (segment 16, Lemma 2).  A 1-D parameter keeps one statistic per segment of
+ * <= b entries, S <- beta2 S + g g^T, rooted at exponent -2/p (full-matrix
+ * Adagrad on the segment when p = 4).
+ *
+ * Conventions for every call below:
+ *  - All work is enqueued, in order, on the CUDA stream given at create time
+ *    and is asynchronous with respect to the host unless a call says that it
+ *    synchronises.
+ *  - Parameters and gradients are CALLER-OWNED device pointers to contiguous
+ *    row-major arrays; the library never frees or keeps them past the call's
+ *    stream work.  Optimizer state (statistics, roots, Adagrad accumulator,
+ *    momentum, work space) is LIBRARY-OWNED device memory, allocated by
+ *    shampoo_create and freed by shampoo_destroy.
+ *  - Errors are returned as a shampoo_status, never by aborting;
+ *    shampoo_last_error() gives a one-line reason.  A context is not
+ *    thread-safe: call it from one host thread at a time.
+ */
+#ifndef SHAMPOO_B200_H
+#define SHAMPOO_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct shampoo_ctx shampoo_ctx;   /* opaque, library-owned */
+
+typedef enum {
+  SHAMPOO_OK = 0,
+  SHAMPOO_EINVAL = 1,         /* bad shape, size, option or null pointer      */
+  SHAMPOO_ENOMEM = 2,         /* device allocation failed                      */
+  SHAMPOO_ECUDA = 3,          /* a CUDA call or kernel launch failed           */
+  SHAMPOO_ENONFINITE = 4,     /* a gradient held NaN/Inf (parameter skipped)   */
+  SHAMPOO_ENOTCONVERGED = 5,  /* some roots did not converge (old roots kept)  */
+  SHAMPOO_ESTATE = 6          /* call out of order (e.g. apply before roots)   */
+} shampoo_status;
+
+typedef enum {
+  SHAMPOO_GRAFT_NONE = 0,     /* U = P                                         */
+  SHAMPOO_GRAFT_ADAGRAD = 1   /* U = (||D||_F / ||P||_F) P per parameter,
+                                 D = g / sqrt(a + eps), a <- beta2 a + g*g     */
+} shampoo_graft;
+
+typedef enum {
+  SHAMPOO_F32 = 0,            /* gradients are float32                         */
+  SHAMPOO_BF16 = 1            /* gradients are bfloat16 (statistics in fp32)   */
+} shampoo_dtype;
+
+/*
+ * shampoo_create -- build the block table and allocate the state.
+ *
+ *  out         receives the new context (set to NULL on failure).
+ *  nparams     number of parameters, >= 1.
+ *  shapes      host array [nparams][2] of (rows, cols), each >= 1.  For a 1-D
+ *              parameter of length n pass (1, n) and set ndims[i] = 1.
+ *  ndims       host array [nparams] of 1 or 2, or NULL for all 2-D.
+ *  block_size  b, the largest block side (segment 16): 64, 128, ..., 1024 (a
+ *              multiple of 64, the tile side of the kernels).  Blocks form a row-major grid from the top-left
+ *              corner; the last block row / column is ragged.
+ *  beta2       statistics decay, 0 < beta2 <= 1 (1 = plain accumulation).
+ *  epsilon     ridge added at root time, (A + eps I)^{-1/p}, and inside the
+ *              graft's sqrt; > 0.
+ *  p           root order for the two factors of a 2-D block (4 in the paper,
+ *              segment 14); 1-D segments use p/2.  p must be 2 or 4.
+ *  graft       SHAMPOO_GRAFT_NONE or SHAMPOO_GRAFT_ADAGRAD (layer-wise).
+ *  momentum    heavy-ball factor mu in [0, 1): m <- mu m + U, W <- W - lr m.
+ *  grad_dtype  element type of every gradient passed later.
+ *  cuda_stream caller-owned cudaStream_t (NULL = legacy default stream).
+ * Statistics, accumulator and momentum start at zero.  Roots start unset;
+ * shampoo_apply fails with SHAMPOO_ESTATE until shampoo_compute_roots ran.
+ * Synchronises the stream once (state zeroing).
+ */
+shampoo_status shampoo_create(shampoo_ctx** out, int nparams,
+                              const int64_t* shapes, const int32_t* ndims,
+                              int block_size, float beta2, float epsilon,
+                              int p, shampoo_graft graft, float momentum,
+                              shampoo_dtype grad_dtype, void* cuda_stream);
+
+/*
+ * shampoo_update_stats -- accumulate gradient outer products (segment 10,
+ * first piece): per block L <- beta2 L + G G^T and R <- beta2 R + G^T G, per
+ * 1-D segment S <- beta2 S + g g^T, and, with grafting, a <- beta2 a + g*g.
+ *  grads  host array [nparams] of device pointers, each to rows*cols
+ *         elements of grad_dtype, row-major.
+ * A parameter whose gradient holds a NaN or Inf is skipped for this step
+ * (statistics, accumulator and, in the next apply, weights and momentum are
+ * left unchanged); the count is read with shampoo_nonfinite_status.
+ */
+shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads);
+
+/*
+ * shampoo_compute_roots -- inverse p-th roots of every statistic (segment
+ * 10, second piece), by the coupled Newton iteration in float64 on the device
+ * (segment 12): X -> (A + eps I)^{-1/p}, stopping per matrix when
+ * max|X^p (A + eps I) - I| <= tol (default 1e-6), giving up on a non-finite
+ * or non-decreasing residual or at the iteration cap (default 100).
+ * The caller picks the interval (segment 14: recompute only now and then).
+ * Synchronises with the host while it runs (it polls the number of matrices
+ * still iterating).  SHAMPOO_ESTATE before the first shampoo_update_stats.
+ * Returns SHAMPOO_ENOTCONVERGED when some matrix gave up:
+ * those keep their previous root (or c^{-1} I, c^p = the eigenvalue bound
+ * the iteration started from, if they never had one); the others are updated.
+ */
+shampoo_status shampoo_compute_roots(shampoo_ctx* ctx);
+
+/*
+ * shampoo_apply -- precondition and update (segment 10, third piece):
+ * per block P = L^{-1/p} G R^{-1/p} (per 1-D segment P = S^{-2/p} g), then
+ * per parameter U = s P with the graft scale s, m <- mu m + U, W <- W - lr m.
+ *  params  host array [nparams] of device float32 pointers, updated in place.
+ *  grads   as for shampoo_update_stats; pass this step's gradients.
+ *  lr      learning rate.
+ * Returns SHAMPOO_ESTATE if roots were never computed.
+ */
+shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params,
+                             const void* const* grads, float lr);
+
+/*
+ * shampoo_root_status -- result of the last shampoo_compute_roots.
+ *  n_not_converged  number of matrices that kept their previous root.
+ *  max_iters        largest Newton iteration count over the matrices.
+ * Either pointer may be NULL.  Host values; synchronises the stream.
+ */
+shampoo_status shampoo_root_status(shampoo_ctx* ctx, int* n_not_converged,
+                                   int* max_iters);
+
+/*
+ * shampoo_nonfinite_status -- number of parameters skipped by the last
+ * shampoo_update_stats because their gradient was not finite.  Synchronises.
+ */
+shampoo_status shampoo_nonfinite_status(shampoo_ctx* ctx, int* n_params_skipped);
+
+/*
+ * shampoo_set_root_options -- Newton stopping rule for later root calls:
+ * tol > 0 on max|M - I|, 1 <= max_iters <= 1000.
+ */
+shampoo_status shampoo_set_root_options(shampoo_ctx* ctx, double tol, int max_iters);
+
+/*
+ * shampoo_num_matrices -- number of statistics matrices: 2 per 2-D block
+ * (L then R, blocks in parameter order, row-major within a parameter), then
+ * 1 per 1-D segment (parameter order).  Each lives in a b x b slot.
+ */
+int shampoo_num_matrices(const shampoo_ctx* ctx);
+
+/*
+ * shampoo_matrix_info -- for statistic `index`: its valid side (the block's
+ * rows for L, columns for R, the segment length for S) and its root exponent
+ * denominator (p, or p/2 for a segment).  Host values.
+ */
+shampoo_status shampoo_matrix_info(const shampoo_ctx* ctx, int index,
+                                   int* size, int* root_p);
+
+/*
+ * shampoo_read_matrix -- copy the b x b float32 slot of statistic `index`
+ * (which = 0) or of its root (which = 1) into dst (host or device memory,
+ * b*b floats, row-major).  Only the top-left size x size corner is the
+ * matrix; the rest is zero.  Synchronises the stream.
+ */
+shampoo_status shampoo_read_matrix(shampoo_ctx* ctx, int which, int index,
+                                   float* dst);
+
+/*
+ * shampoo_root_iterations -- per-matrix Newton iteration counts of the last
+ * shampoo_compute_roots, in statistic order: k >= 0 when matrix i converged
+ * after k steps, -1-k when it gave up at step k.
+ *  out  host array of shampoo_num_matrices(ctx) int32 values.
+ * SHAMPOO_ESTATE before the first shampoo_compute_roots.
+ */
+shampoo_status shampoo_root_iterations(shampoo_ctx* ctx, int32_t* out);
+
+/*
+ * Kernel profiling.  The library counts every kernel it launches, per
+ * kernel name.  With profiling enabled it also records a pair of CUDA events
+ * on the context's stream around each launch and sums their elapsed times.
+ *  shampoo_profile_enable  clears the counters; on != 0 turns event timing on.
+ *  shampoo_profile_count   number of kernel names seen since the last enable.
+ *  shampoo_profile_entry   for name `index`: the name (copied into name, at
+ *                          most name_len bytes with the terminating NUL), the
+ *                          launch count and the summed milliseconds (0 when
+ *                          timing was off).  Synchronises on pending events.
+ */
+shampoo_status shampoo_profile_enable(shampoo_ctx* ctx, int on);
+int shampoo_profile_count(const shampoo_ctx* ctx);
+shampoo_status shampoo_profile_entry(shampoo_ctx* ctx, int index, char* name, int name_len,
+                                     int64_t* launches, double* ms);
+
+/*
+ * shampoo_last_error -- one-line reason for the last failed call on ctx
+ * (empty string if none).  ctx may be NULL for a create failure.
+ */
+const char* shampoo_last_error(const shampoo_ctx* ctx);
+
+/* shampoo_destroy -- free all library-owned memory.  NULL is a no-op. */
+void shampoo_destroy(shampoo_ctx* ctx);
+
+/*
+ * shampoo_batched_inverse_root -- the root kernel on its own (segment 12):
+ * X_i = (A_i + eps I)^{-1/p} for `batch` symmetric PSD n x n matrices, by
+ * coupled Newton in float64 on the device.
+ *  A       device float32 [batch][n][n], row-major, symmetric (read only).
+ *  X       device float32 [batch][n][n] output (caller-owned).
+ *  batch   >= 1;  n in [1, 1024];  p in {2, 4};  eps > 0;  tol > 0;
+ *  max_iters in [1, 1000].
+ *  iters   device int32 [batch] or NULL: per-matrix iteration count k, or
+ *          -1-k when the matrix gave up at iteration k.  On give-up X_i holds
+ *          c^{-1} I (c^p = the starting eigenvalue bound).
+ *  stream  caller-owned cudaStream_t.
+ * Allocates its float64 work space (6 n x n per matrix in flight, at most
+ * 2 GiB) with cudaMalloc and frees it before returning.  Synchronises while it
+ * runs, like shampoo_compute_roots.  Returns SHAMPOO_ENOTCONVERGED if any
+ * matrix gave up.
+ */
+shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
+                                            int n, int p, float eps, double tol,
+                                            int max_iters, int32_t* iters,
+                                            void* stream);
+
+/* Library version, "MAJOR.MINOR.PATCH". */
+const char* shampoo_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHAMPOO_B200_H */

@@ -1,0 +1,645 @@
+// C-ABI of the library (include/shampoo.h): the host-side planner that builds
+// the block table, owns the device state and sequences the kernels of one
+// optimizer step on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/shampoo.h"
+#include "internal.h"
+
+using namespace shampoo;
+
+namespace {
+
+// Per-kernel launch counts and, when enabled, CUDA-event times taken on the
+// caller's stream around each launch.
+struct Profiler {
+  struct Entry {
+    std::string name;
+    int64_t launches = 0;
+    double ms = 0.0;
+  };
+  struct Pending {
+    int entry;
+    cudaEvent_t a, b;
+  };
+  bool on = false;
+  std::vector<Entry> entries;
+  std::vector<Pending> pending;
+  std::vector<cudaEvent_t> pool;
+
+  int find(const char* name) {
+    for (size_t i = 0; i < entries.size(); ++i)
+      if (entries[i].name == name) return (int)i;
+    entries.push_back(Entry{name, 0, 0.0});
+    return (int)entries.size() - 1;
+  }
+  cudaEvent_t event() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  template <class F>
+  void launch(const char* name, cudaStream_t s, F&& f) {
+    const int e = find(name);
+    ++entries[e].launches;
+    if (!on) {
+      f();
+      return;
+    }
+    cudaEvent_t a = event(), b = event();
+    cudaEventRecord(a, s);
+    f();
+    cudaEventRecord(b, s);
+    pending.push_back(Pending{e, a, b});
+  }
+  cudaError_t flush() {
+    cudaError_t err = cudaSuccess;
+    for (auto& p : pending) {
+      float ms = 0.f;
+      cudaError_t e = cudaEventSynchronize(p.b);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, p.a, p.b);
+      if (e != cudaSuccess) err = e;
+      entries[p.entry].ms += ms;
+      pool.push_back(p.a);
+      pool.push_back(p.b);
+    }
+    pending.clear();
+    return err;
+  }
+  void reset() {
+    flush();
+    entries.clear();
+  }
+  ~Profiler() {
+    flush();
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+
+// Launch through the profiler when there is one.
+template <class F>
+void run(Profiler* pr, const char* name, cudaStream_t s, F&& f) {
+  if (pr) pr->launch(name, s, f);
+  else f();
+}
+
+}  // namespace
+
+struct shampoo_ctx {
+  cudaStream_t stream = nullptr;
+  int nparams = 0, b = 0, S = 0, p = 4, graft = 1, bf16 = 0;
+  float beta2 = 1.f, eps = 1e-6f, mu = 0.f;
+  double tol = 1e-6;
+  int max_iters = 100;
+
+  std::vector<ParamDesc> params;
+  std::vector<int> ndim;
+  std::vector<BlockDesc> blocks;
+  std::vector<SegDesc> segs;
+  std::vector<ChunkDesc> chunks;
+  std::vector<NewtonMat> mats;
+  int64_t total = 0;
+  int nmat = 0;
+
+  // device
+  ParamDesc* d_params = nullptr;
+  BlockDesc* d_blocks = nullptr;
+  SegDesc* d_segs = nullptr;
+  ChunkDesc* d_chunks = nullptr;
+  NewtonMat* d_mats = nullptr;
+  const void** d_gptr = nullptr;
+  float** d_wptr = nullptr;
+  float* stats = nullptr;
+  float* roots = nullptr;
+  float* a = nullptr;
+  float* mom = nullptr;
+  float* P = nullptr;
+  float* Y = nullptr;
+  double* norms = nullptr;
+  int* flags = nullptr;
+  int* has_root = nullptr;
+  NewtonWork nw{};
+  int newton_chunk = 0;
+  int* h_count = nullptr;   // pinned [2]
+  cudaEvent_t ev[2] = {nullptr, nullptr};
+  std::vector<void*> allocs;
+
+  bool stats_done = false, roots_done = false;
+  int last_not_converged = 0, last_max_iters = 0;
+  std::vector<int32_t> root_iters;   // per matrix, last compute_roots (-1-k: gave up at k)
+  Profiler prof;
+  std::string err;
+};
+
+namespace {
+
+thread_local std::string g_create_err;
+
+shampoo_status fail(shampoo_ctx* c, shampoo_status st, const std::string& msg) {
+  if (c) c->err = msg; else g_create_err = msg;
+  return st;
+}
+
+shampoo_status cuda_fail(shampoo_ctx* c, cudaError_t e, const char* what) {
+  return fail(c, SHAMPOO_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(call)                                               \
+  do {                                                         \
+    cudaError_t e_ = (call);                                   \
+    if (e_ != cudaSuccess) return cuda_fail(ctx, e_, #call);   \
+  } while (0)
+
+template <class T>
+cudaError_t dalloc(shampoo_ctx* ctx, T** p, size_t count) {
+  *p = nullptr;
+  if (count == 0) return cudaSuccess;
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, count * sizeof(T));
+  if (e == cudaSuccess) {
+    ctx->allocs.push_back(q);
+    *p = static_cast<T*>(q);
+  }
+  return e;
+}
+
+template <class T>
+shampoo_status upload(shampoo_ctx* ctx, T** dst, const std::vector<T>& v) {
+  cudaError_t e = dalloc(ctx, dst, v.size());
+  if (e != cudaSuccess) return fail(ctx, SHAMPOO_ENOMEM, "cudaMalloc of the block table failed");
+  if (!v.empty()) CK(cudaMemcpy(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice));
+  return SHAMPOO_OK;
+}
+
+// Newton work space for `chunk` matrices of side S.
+cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
+  const size_t mat = (size_t)chunk * S * S;
+  cudaError_t e = cudaSuccess;
+  double** bufs[7] = {&w.X[0], &w.X[1], &w.M[0], &w.M[1], &w.T, &w.T2, &w.T4};
+  for (auto b : bufs)
+    if ((e = dalloc(ctx, b, mat)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.cinv, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.resid, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.prev, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.worse, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.iters, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.state, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.count, 2)) != cudaSuccess) return e;
+  return e;
+}
+
+// Run the Newton iteration over mats[0..nm) (device array dm) in chunks of
+// `chunk` matrices.  A/X are float32 slot arrays.  Returns the number of
+// matrices that gave up and the largest iteration count through outs.
+shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<NewtonMat>& hm,
+                          const NewtonMat* dm, const float* A, int64_t a_stride, int lda, float* X,
+                          int64_t x_stride, int ldx, int S, float eps, double tol, int max_iters,
+                          int chunk, NewtonWork& w, int* has_root, int32_t* iters_out, int* h_count,
+                          cudaEvent_t* ev, cudaStream_t st, int* n_failed, int* max_it,
+                          std::vector<int32_t>* per_matrix) {
+  *n_failed = 0;
+  *max_it = 0;
+  const int nm_all = (int)hm.size();
+  if (per_matrix) per_matrix->assign(nm_all, 0);
+  std::vector<int> hstate(chunk), hiters(chunk);
+  for (int c0 = 0; c0 < nm_all; c0 += chunk) {
+    const int nm = std::min(chunk, nm_all - c0);
+    const NewtonMat* d = dm + c0;
+    int has_p4 = 0;
+    for (int i = 0; i < nm; ++i) has_p4 |= (hm[c0 + i].p == 4);
+    run(pr, "newton_reset", st, [&] { launch_newton_reset(nm, w, st); });
+    run(pr, "newton_bound", st, [&] { launch_newton_bound(A, a_stride, lda, d, nm, eps, w, st); });
+    run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, d, nm, S, eps, w, st); });
+    run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
+    CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
+    CK(cudaEventRecord(ev[0], st));
+    for (int it = 0; it < max_iters; ++it) {
+      // the check of M_it is in flight; queue step it+1 before waiting for it
+      run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, w, st); });
+      if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, w, st); });
+      run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, w, st); });
+      run(pr, "newton_check", st, [&] { launch_newton_check(nm, it + 1, tol, max_iters, w, st); });
+      const int nx = (it + 1) & 1;
+      CK(cudaGetLastError());
+      CK(cudaMemcpyAsync(&h_count[nx], &w.count[nx], sizeof(int), cudaMemcpyDeviceToHost, st));
+      CK(cudaEventRecord(ev[nx], st));
+      CK(cudaEventSynchronize(ev[it & 1]));
+      if (h_count[it & 1] == 0) break;
+    }
+    run(pr, "newton_finalize", st, [&] {
+      launch_newton_finalize(X, x_stride, ldx, d, nm, S, w, has_root, iters_out, st);
+    });
+    CK(cudaGetLastError());
+    CK(cudaMemcpyAsync(hstate.data(), w.state, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(hiters.data(), w.iters, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    for (int i = 0; i < nm; ++i) {
+      if (hstate[i] != 1) ++*n_failed;
+      *max_it = std::max(*max_it, hiters[i]);
+      if (per_matrix) (*per_matrix)[c0 + i] = hstate[i] == 1 ? hiters[i] : -1 - hiters[i];
+    }
+  }
+  return SHAMPOO_OK;
+}
+
+shampoo_status set_pointers(shampoo_ctx* ctx, const void* const* grads, float* const* params) {
+  if (!grads) return fail(ctx, SHAMPOO_EINVAL, "grads is NULL");
+  for (int i = 0; i < ctx->nparams; ++i)
+    if (!grads[i]) return fail(ctx, SHAMPOO_EINVAL, "grads[" + std::to_string(i) + "] is NULL");
+  // pageable source: staged by the driver before the call returns
+  CK(cudaMemcpyAsync(ctx->d_gptr, grads, ctx->nparams * sizeof(void*), cudaMemcpyHostToDevice,
+                     ctx->stream));
+  if (params) {
+    for (int i = 0; i < ctx->nparams; ++i)
+      if (!params[i]) return fail(ctx, SHAMPOO_EINVAL, "params[" + std::to_string(i) + "] is NULL");
+    CK(cudaMemcpyAsync(ctx->d_wptr, params, ctx->nparams * sizeof(float*), cudaMemcpyHostToDevice,
+                       ctx->stream));
+  }
+  return SHAMPOO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* shampoo_version(void) { return "0.1.0"; }
+
+const char* shampoo_last_error(const shampoo_ctx* ctx) {
+  return ctx ? ctx->err.c_str() : g_create_err.c_str();
+}
+
+void shampoo_destroy(shampoo_ctx* ctx) {
+  if (!ctx) return;
+  cudaStreamSynchronize(ctx->stream);
+  for (void* q : ctx->allocs) cudaFree(q);
+  if (ctx->h_count) cudaFreeHost(ctx->h_count);
+  for (auto& e : ctx->ev)
+    if (e) cudaEventDestroy(e);
+  delete ctx;
+}
+
+shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* shapes,
+                              const int32_t* ndims, int block_size, float beta2, float epsilon,
+                              int p, shampoo_graft graft, float momentum, shampoo_dtype grad_dtype,
+                              void* cuda_stream) {
+  if (!out) return fail(nullptr, SHAMPOO_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (nparams < 1 || !shapes) return fail(nullptr, SHAMPOO_EINVAL, "need nparams >= 1 and shapes");
+  if (block_size < 64 || block_size > 1024 || block_size % 64)
+    return fail(nullptr, SHAMPOO_EINVAL, "block_size must be a multiple of 64 in [64, 1024]");
+  if (!(beta2 > 0.f && beta2 <= 1.f)) return fail(nullptr, SHAMPOO_EINVAL, "beta2 must be in (0, 1]");
+  if (!(epsilon > 0.f) || !std::isfinite(epsilon)) return fail(nullptr, SHAMPOO_EINVAL, "epsilon must be > 0");
+  if (p != 2 && p != 4) return fail(nullptr, SHAMPOO_EINVAL, "p must be 2 or 4");
+  if (graft != SHAMPOO_GRAFT_NONE && graft != SHAMPOO_GRAFT_ADAGRAD)
+    return fail(nullptr, SHAMPOO_EINVAL, "unknown graft");
+  if (!(momentum >= 0.f && momentum < 1.f)) return fail(nullptr, SHAMPOO_EINVAL, "momentum must be in [0, 1)");
+  if (grad_dtype != SHAMPOO_F32 && grad_dtype != SHAMPOO_BF16)
+    return fail(nullptr, SHAMPOO_EINVAL, "unknown grad dtype");
+
+  shampoo_ctx* ctx = new shampoo_ctx();
+  ctx->stream = static_cast<cudaStream_t>(cuda_stream);
+  ctx->nparams = nparams;
+  ctx->b = ctx->S = block_size;
+  ctx->p = p;
+  ctx->beta2 = beta2;
+  ctx->eps = epsilon;
+  ctx->mu = momentum;
+  ctx->graft = graft;
+  ctx->bf16 = grad_dtype == SHAMPOO_BF16;
+  const int b = block_size;
+
+  for (int i = 0; i < nparams; ++i) {
+    const int64_t r = shapes[2 * i], c = shapes[2 * i + 1];
+    const int nd = ndims ? ndims[i] : 2;
+    if (r < 1 || c < 1 || (nd != 1 && nd != 2) || (nd == 1 && r != 1) || r > (1ll << 31) ||
+        c > (1ll << 31)) {
+      delete ctx;
+      return fail(nullptr, SHAMPOO_EINVAL, "bad shape or ndim for parameter " + std::to_string(i));
+    }
+    ParamDesc pd;
+    pd.numel = r * c;
+    pd.offset = ctx->total;
+    ctx->total += (pd.numel + 3) & ~int64_t(3);   // 16-byte aligned parameter starts
+    ctx->params.push_back(pd);
+    ctx->ndim.push_back(nd);
+    if (nd == 2) {
+      for (int64_t r0 = 0; r0 < r; r0 += b)
+        for (int64_t c0 = 0; c0 < c; c0 += b) {
+          BlockDesc bd;
+          bd.param = i;
+          bd.r0 = r0;
+          bd.c0 = c0;
+          bd.m = (int)std::min<int64_t>(b, r - r0);
+          bd.n = (int)std::min<int64_t>(b, c - c0);
+          bd.ld = c;
+          ctx->blocks.push_back(bd);
+        }
+    }
+    for (int64_t s0 = 0; s0 < pd.numel; s0 += kChunk) {
+      ChunkDesc ch;
+      ch.param = i;
+      ch.start = s0;
+      ch.len = (int)std::min<int64_t>(kChunk, pd.numel - s0);
+      ctx->chunks.push_back(ch);
+    }
+  }
+  for (int i = 0; i < nparams; ++i) {
+    if (ctx->ndim[i] != 1) continue;
+    for (int64_t s0 = 0; s0 < ctx->params[i].numel; s0 += b) {
+      SegDesc sd;
+      sd.param = i;
+      sd.s0 = s0;
+      sd.len = (int)std::min<int64_t>(b, ctx->params[i].numel - s0);
+      ctx->segs.push_back(sd);
+    }
+  }
+  for (size_t k = 0; k < ctx->blocks.size(); ++k) {
+    ctx->mats.push_back({(int)(2 * k), ctx->blocks[k].m, p, 0});
+    ctx->mats.push_back({(int)(2 * k + 1), ctx->blocks[k].n, p, 0});
+  }
+  const int mat0 = 2 * (int)ctx->blocks.size();
+  for (size_t k = 0; k < ctx->segs.size(); ++k)
+    ctx->mats.push_back({mat0 + (int)k, ctx->segs[k].len, p / 2, 0});
+  ctx->nmat = (int)ctx->mats.size();
+
+  shampoo_status st;
+  if ((st = upload(ctx, &ctx->d_params, ctx->params)) != SHAMPOO_OK ||
+      (st = upload(ctx, &ctx->d_blocks, ctx->blocks)) != SHAMPOO_OK ||
+      (st = upload(ctx, &ctx->d_segs, ctx->segs)) != SHAMPOO_OK ||
+      (st = upload(ctx, &ctx->d_chunks, ctx->chunks)) != SHAMPOO_OK ||
+      (st = upload(ctx, &ctx->d_mats, ctx->mats)) != SHAMPOO_OK) {
+    g_create_err = ctx->err;
+    shampoo_destroy(ctx);
+    return st;
+  }
+  const size_t slot = (size_t)b * b;
+  // Newton work space: at most ~4 GiB of float64 in flight.
+  const size_t per = 7 * slot * sizeof(double);
+  ctx->newton_chunk = (int)std::max<size_t>(1, std::min<size_t>(ctx->nmat, (size_t(4) << 30) / per));
+  cudaError_t e = cudaSuccess;
+  bool okm = (e = dalloc(ctx, &ctx->d_gptr, nparams)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->d_wptr, nparams)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->stats, ctx->nmat * slot)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->roots, ctx->nmat * slot)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->a, (size_t)ctx->total)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->P, (size_t)ctx->total)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->Y, ctx->blocks.size() * slot)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->norms, 2 * (size_t)nparams)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->flags, (size_t)nparams)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->has_root, (size_t)ctx->nmat)) == cudaSuccess &&
+             (momentum == 0.f || (e = dalloc(ctx, &ctx->mom, (size_t)ctx->total)) == cudaSuccess) &&
+             (e = alloc_newton(ctx, ctx->nw, ctx->newton_chunk, b)) == cudaSuccess;
+  if (!okm) {
+    shampoo_destroy(ctx);
+    return fail(nullptr, SHAMPOO_ENOMEM, std::string("device allocation failed: ") + cudaGetErrorString(e));
+  }
+  e = cudaMallocHost(&ctx->h_count, 2 * sizeof(int));
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->stats, 0, ctx->nmat * slot * sizeof(float), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->roots, 0, ctx->nmat * slot * sizeof(float), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->a, 0, ctx->total * sizeof(float), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->P, 0, ctx->total * sizeof(float), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->flags, 0, nparams * sizeof(int), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->has_root, 0, ctx->nmat * sizeof(int), ctx->stream);
+  if (e == cudaSuccess && ctx->mom) e = cudaMemsetAsync(ctx->mom, 0, ctx->total * sizeof(float), ctx->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
+  if (e != cudaSuccess) {
+    shampoo_destroy(ctx);
+    return fail(nullptr, SHAMPOO_ECUDA, std::string("state set-up failed: ") + cudaGetErrorString(e));
+  }
+  *out = ctx;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  shampoo_status st = set_pointers(ctx, grads, nullptr);
+  if (st != SHAMPOO_OK) return st;
+  cudaStream_t s = ctx->stream;
+  const int nch = (int)ctx->chunks.size();
+  const int nblk = (int)ctx->blocks.size(), nseg = (int)ctx->segs.size();
+  Profiler* pr = &ctx->prof;
+  CK(cudaMemsetAsync(ctx->flags, 0, ctx->nparams * sizeof(int), s));
+  run(pr, "check_finite", s, [&] {
+    launch_check_finite(ctx->d_chunks, nch, ctx->d_gptr, ctx->bf16, ctx->flags, s);
+  });
+  if (ctx->graft)
+    run(pr, "diag_update", s, [&] {
+      launch_diag_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags,
+                         ctx->beta2, ctx->a, s);
+    });
+  if (nblk)
+    run(pr, "stats_blocks", s, [&] {
+      launch_stats_blocks(ctx->d_blocks, nblk, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->beta2,
+                          ctx->stats, ctx->S, s);
+    });
+  if (nseg)
+    run(pr, "stats_segments", s, [&] {
+      launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
+                            ctx->beta2, ctx->stats, ctx->S, s);
+    });
+  CK(cudaGetLastError());
+  ctx->stats_done = true;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  int nf = 0, mi = 0;
+  if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots before update_stats");
+  const int64_t slot = (int64_t)ctx->S * ctx->S;
+  shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->stats, slot, ctx->S,
+                                 ctx->roots, slot, ctx->S, ctx->S, ctx->eps, ctx->tol,
+                                 ctx->max_iters, ctx->newton_chunk, ctx->nw, ctx->has_root, nullptr,
+                                 ctx->h_count, ctx->ev, ctx->stream, &nf, &mi, &ctx->root_iters);
+  if (st != SHAMPOO_OK) return st;
+  ctx->roots_done = true;
+  ctx->last_not_converged = nf;
+  ctx->last_max_iters = mi;
+  if (nf) return fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void* const* grads,
+                             float lr) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (!ctx->roots_done) return fail(ctx, SHAMPOO_ESTATE, "apply before compute_roots");
+  if (!params) return fail(ctx, SHAMPOO_EINVAL, "params is NULL");
+  shampoo_status st = set_pointers(ctx, grads, params);
+  if (st != SHAMPOO_OK) return st;
+  cudaStream_t s = ctx->stream;
+  const int nch = (int)ctx->chunks.size();
+  const int nblk = (int)ctx->blocks.size();
+  const int nseg = (int)ctx->segs.size();
+  Profiler* pr = &ctx->prof;
+  CK(cudaMemsetAsync(ctx->norms, 0, 2 * ctx->nparams * sizeof(double), s));
+  if (ctx->graft)
+    run(pr, "dnorm", s, [&] {
+      launch_dnorm(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->a,
+                   ctx->eps, ctx->norms, s);
+    });
+  if (nblk) {
+    run(pr, "precond_y", s, [&] {
+      launch_precond_y(ctx->d_blocks, nblk, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->roots, ctx->S,
+                       ctx->Y, s);
+    });
+    run(pr, "precond_p", s, [&] {
+      launch_precond_p(ctx->d_blocks, nblk, ctx->d_params, ctx->flags, ctx->roots, ctx->S, ctx->Y,
+                       ctx->P, ctx->norms, s);
+    });
+  }
+  if (nseg)
+    run(pr, "precond_seg", s, [&] {
+      launch_precondition_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_params, ctx->d_gptr,
+                                   ctx->bf16, ctx->flags, ctx->roots, ctx->S, ctx->P, ctx->norms, s);
+    });
+  run(pr, "update", s, [&] {
+    launch_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_wptr, ctx->flags, ctx->P, ctx->norms,
+                  ctx->graft, ctx->mu, lr, ctx->mom, s);
+  });
+  CK(cudaGetLastError());
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_root_status(shampoo_ctx* ctx, int* n_not_converged, int* max_iters) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  CK(cudaStreamSynchronize(ctx->stream));
+  if (n_not_converged) *n_not_converged = ctx->last_not_converged;
+  if (max_iters) *max_iters = ctx->last_max_iters;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_nonfinite_status(shampoo_ctx* ctx, int* n_params_skipped) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (!n_params_skipped) return fail(ctx, SHAMPOO_EINVAL, "n_params_skipped is NULL");
+  std::vector<int> f(ctx->nparams);
+  CK(cudaMemcpyAsync(f.data(), ctx->flags, ctx->nparams * sizeof(int), cudaMemcpyDeviceToHost,
+                     ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  int n = 0;
+  for (int v : f) n += v != 0;
+  *n_params_skipped = n;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_set_root_options(shampoo_ctx* ctx, double tol, int max_iters) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (!(tol > 0.0) || max_iters < 1 || max_iters > 1000)
+    return fail(ctx, SHAMPOO_EINVAL, "need tol > 0 and 1 <= max_iters <= 1000");
+  ctx->tol = tol;
+  ctx->max_iters = max_iters;
+  return SHAMPOO_OK;
+}
+
+int shampoo_num_matrices(const shampoo_ctx* ctx) { return ctx ? ctx->nmat : 0; }
+
+shampoo_status shampoo_matrix_info(const shampoo_ctx* ctx, int index, int* size, int* root_p) {
+  if (!ctx || index < 0 || index >= ctx->nmat) return SHAMPOO_EINVAL;
+  if (size) *size = ctx->mats[index].size;
+  if (root_p) *root_p = ctx->mats[index].p;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_read_matrix(shampoo_ctx* ctx, int which, int index, float* dst) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if ((which != 0 && which != 1) || index < 0 || index >= ctx->nmat || !dst)
+    return fail(ctx, SHAMPOO_EINVAL, "bad which / index / dst");
+  const size_t slot = (size_t)ctx->S * ctx->S;
+  const float* src = (which == 0 ? ctx->stats : ctx->roots) + slot * index;
+  CK(cudaMemcpyAsync(dst, src, slot * sizeof(float), cudaMemcpyDefault, ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_root_iterations(shampoo_ctx* ctx, int32_t* out) {
+  if (!ctx || !out) return fail(ctx, SHAMPOO_EINVAL, "ctx or out is NULL");
+  if (ctx->root_iters.empty()) return fail(ctx, SHAMPOO_ESTATE, "no roots computed yet");
+  std::memcpy(out, ctx->root_iters.data(), ctx->root_iters.size() * sizeof(int32_t));
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_profile_enable(shampoo_ctx* ctx, int on) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  ctx->prof.reset();
+  ctx->prof.on = on != 0;
+  return SHAMPOO_OK;
+}
+
+int shampoo_profile_count(const shampoo_ctx* ctx) { return ctx ? (int)ctx->prof.entries.size() : 0; }
+
+shampoo_status shampoo_profile_entry(shampoo_ctx* ctx, int index, char* name, int name_len,
+                                     int64_t* launches, double* ms) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  CK(ctx->prof.flush());
+  if (index < 0 || index >= (int)ctx->prof.entries.size())
+    return fail(ctx, SHAMPOO_EINVAL, "profile index out of range");
+  const auto& e = ctx->prof.entries[index];
+  if (name && name_len > 0) {
+    std::strncpy(name, e.name.c_str(), name_len - 1);
+    name[name_len - 1] = 0;
+  }
+  if (launches) *launches = e.launches;
+  if (ms) *ms = e.ms;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch, int n, int p,
+                                            float eps, double tol, int max_iters, int32_t* iters,
+                                            void* stream) {
+  if (!A || !X || batch < 1 || n < 1 || n > 1024 || (p != 2 && p != 4) || !(eps > 0.f) ||
+      !(tol > 0.0) || max_iters < 1 || max_iters > 1000)
+    return fail(nullptr, SHAMPOO_EINVAL, "bad argument to shampoo_batched_inverse_root");
+  shampoo_ctx tmp;   // carries the allocations and the error text only
+  shampoo_ctx* ctx = &tmp;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int S = (n + kTile - 1) / kTile * kTile;
+  const size_t per = 7 * (size_t)S * S * sizeof(double);
+  const int chunk = (int)std::max<size_t>(1, std::min<size_t>(batch, (size_t(2) << 30) / per));
+  std::vector<NewtonMat> hm(batch);
+  for (int i = 0; i < batch; ++i) hm[i] = {i, n, p, 0};
+  NewtonMat* dm = nullptr;
+  NewtonWork w{};
+  shampoo_status res = SHAMPOO_OK;
+  int nf = 0, mi = 0;
+  cudaError_t e = cudaSuccess;
+  if ((res = upload(ctx, &dm, hm)) != SHAMPOO_OK) goto done;
+  if ((e = alloc_newton(ctx, w, chunk, S)) != cudaSuccess) {
+    res = fail(ctx, SHAMPOO_ENOMEM, std::string("work space: ") + cudaGetErrorString(e));
+    goto done;
+  }
+  if ((e = cudaMallocHost(&ctx->h_count, 2 * sizeof(int))) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming)) != cudaSuccess) {
+    res = cuda_fail(ctx, e, "set-up");
+    goto done;
+  }
+  res = run_newton(ctx, nullptr, hm, dm, A, (int64_t)n * n, n, X, (int64_t)n * n, n, S, eps, tol,
+                   max_iters, chunk, w, nullptr, iters, ctx->h_count, ctx->ev, st, &nf, &mi, nullptr);
+  if (res == SHAMPOO_OK && nf) res = fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
+done:
+  cudaStreamSynchronize(st);
+  for (void* q : ctx->allocs) cudaFree(q);
+  ctx->allocs.clear();
+  if (ctx->h_count) cudaFreeHost(ctx->h_count);
+  ctx->h_count = nullptr;
+  for (auto& ev : ctx->ev)
+    if (ev) cudaEventDestroy(ev);
+  ctx->ev[0] = ctx->ev[1] = nullptr;
+  if (res != SHAMPOO_OK) g_create_err = ctx->err;
+  return res;
+}
+
+}  // extern "C"

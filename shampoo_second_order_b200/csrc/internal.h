@@ -1,0 +1,111 @@
+// Internal declarations shared by the host planner and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace shampoo {
+
+// One 2-D block of a parameter (a <= b x b tile of the row-major grid).
+struct BlockDesc {
+  int param;     // parameter index
+  int m, n;      // valid rows / cols of the block
+  int64_t r0, c0;  // top-left element in the parameter
+  int64_t ld;    // the parameter's row length (cols)
+};
+
+// One segment of a 1-D parameter.
+struct SegDesc {
+  int param;
+  int len;
+  int64_t s0;
+};
+
+// A contiguous run of one parameter's elements, the unit of the elementwise
+// kernels (Adagrad accumulator, graft norms, weight update).
+struct ChunkDesc {
+  int param;
+  int len;
+  int64_t start;   // element offset inside the parameter
+};
+
+struct ParamDesc {
+  int64_t numel;
+  int64_t offset;  // element offset into the flat parameter-shaped buffers
+};
+
+constexpr int kChunk = 16384;   // elements per elementwise chunk
+constexpr int kTile = 64;       // tile side of every matrix kernel
+
+// Per-matrix bookkeeping of the Newton root iteration.
+struct NewtonMat {
+  int slot;        // statistic slot (stats / roots arrays)
+  int size;        // valid side
+  int p;           // root order
+  int pad;
+};
+
+// ---------------- stats (k_stats.cu) ----------------
+void launch_check_finite(const ChunkDesc* chunks, int nchunks, const void* const* gptr,
+                         int bf16, int* flags, cudaStream_t s);
+void launch_diag_update(const ChunkDesc* chunks, int nchunks, const ParamDesc* params,
+                        const void* const* gptr, int bf16, const int* flags, float beta2,
+                        float* a, cudaStream_t s);
+void launch_stats_blocks(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
+                         const int* flags, float beta2, float* stats, int S, cudaStream_t s);
+void launch_stats_segments(const SegDesc* segs, int nseg, int mat0, const void* const* gptr,
+                           int bf16, const int* flags, float beta2, float* stats, int S,
+                           cudaStream_t s);
+
+// ---------------- roots (k_roots.cu) ----------------
+struct NewtonWork {
+  double* X[2];
+  double* M[2];
+  double* T;
+  double* T2;
+  double* T4;
+  double* cinv;                 // [nmat] c^{-1}
+  unsigned long long* resid;    // [nmat] max|M-I| as ordered bits
+  double* prev;                 // [nmat] previous residual
+  int* worse;                   // [nmat]
+  int* active;                  // [nmat]
+  int* iters;                   // [nmat] iterations done
+  int* state;                   // [nmat] 0 running, 1 converged, 2 failed
+  int* count;                   // [1] matrices still active after a check
+};
+// Set up X0, M0, T0 for `nm` matrices read from `A` (float32, slot-strided
+// `a_stride` elements apart, row stride `lda`, valid side mats[i].size).
+void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s);
+void launch_newton_bound(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
+                         float eps, NewtonWork w, cudaStream_t s);
+void launch_newton_init(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
+                        int S, float eps, NewtonWork w, cudaStream_t s);
+// one Newton step: A (X T and T T), B (T2 T2, p = 4 only), C (T^p M,
+// residual, next T); check k: convergence test of M_k
+void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);
+void launch_newton_step_b(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
+void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);
+void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s);
+// Write the roots back as float32.  keep_old: leave a failed matrix's slot
+// untouched if has_root[slot] is set; else write c^{-1} I.
+void launch_newton_finalize(float* X, int64_t x_stride, int ldx, const NewtonMat* mats, int nm,
+                            int S, NewtonWork w, int* has_root, int32_t* iters_out,
+                            cudaStream_t s);
+
+// ---------------- apply (k_apply.cu) ----------------
+void launch_dnorm(const ChunkDesc* chunks, int nchunks, const ParamDesc* params,
+                  const void* const* gptr, int bf16, const int* flags, const float* a, float eps,
+                  double* norms, cudaStream_t s);
+void launch_precond_y(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
+                      const int* flags, const float* roots, int S, float* Y, cudaStream_t s);
+void launch_precond_p(const BlockDesc* blocks, int nblk, const ParamDesc* params, const int* flags,
+                      const float* roots, int S, const float* Y, float* P, double* norms,
+                      cudaStream_t s);
+void launch_precondition_segments(const SegDesc* segs, int nseg, int mat0, const ParamDesc* params,
+                                  const void* const* gptr, int bf16, const int* flags,
+                                  const float* roots, int S, float* P, double* norms,
+                                  cudaStream_t s);
+void launch_update(const ChunkDesc* chunks, int nchunks, const ParamDesc* params, float* const* wptr,
+                   const int* flags, const float* P, const double* norms, int graft, float mu,
+                   float lr, float* mom, cudaStream_t s);
+
+}  // namespace shampoo

@@ -1,0 +1,399 @@
+// Batched inverse p-th roots by the coupled Newton iteration in float64
+// (transcript segment 12: the root must be taken in double precision; this
+// is the coupled Newton iteration it names, Guo & Higham 2006):
+//
+//   c^p >= lambda_max(A + eps I),  X0 = c^{-1} I,  M0 = (A + eps I) / c^p
+//   T = ((p+1) I - M) / p,  X <- X T,  M <- T^p M,   until max|M - I| <= tol
+//
+// Every matrix the iteration touches is a polynomial in A, so all of them are
+// symmetric and commute: each product is computed on the upper-triangular
+// 64 x 64 tiles only and written to both (i, j) and (j, i).  The products run
+// on the float64 tensor-core MMA (mma.sync m8n8k4 .f64).  A ragged statistic
+// sits in the top-left corner of its S x S slot; the padding is set to the
+// identity in M (so T = I there) and never mixes with the valid corner.
+#include <float.h>
+
+#include "common.cuh"
+
+namespace shampoo {
+
+namespace {
+
+constexpr int kNewtonThreads = 128;
+constexpr int kBK = 16;
+constexpr int kAStride = kBK + 4;     // doubles; 4 mod 16 keeps fragment loads conflict-free
+constexpr int kBStride = kTile + 4;
+
+enum : int { kRunning = 0, kConverged = 1, kFailed = 2 };
+
+__device__ __forceinline__ unsigned long long dbl_bits(double v) {
+  return static_cast<unsigned long long>(__double_as_longlong(v));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void dmma884(double& c0, double& c1, double a, double b) {
+  asm volatile(
+      "mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+      : "+d"(c0), "+d"(c1)
+      : "d"(a), "d"(b));
+}
+
+// Tile (ti, tj) of the upper triangle of a T x T tile grid, from its index.
+__device__ __forceinline__ void tri_tile(int idx, int T, int& ti, int& tj) {
+  ti = 0;
+  while (idx >= T - ti) {
+    idx -= T - ti;
+    ++ti;
+  }
+  tj = ti + idx;
+}
+
+struct NewtonSmem {
+  double As[2][kTile][kAStride];
+  double Bs[2][kBK][kBStride];
+};
+
+// acc = A[i0:i0+64, :] * B[:, j0:j0+64] for S x S row-major float64 A, B.
+// 4 warps in a 2 x 2 arrangement, each a 32 x 32 sub-tile of 4 x 4 m8n8
+// fragments; lane (g, t) = (lane / 4, lane % 4) holds acc[mi][ni][e] at row
+// 8 mi + g, column 8 ni + 2 t + e of its sub-tile.
+__device__ __forceinline__ void dmma_tile(const double* __restrict__ A, const double* __restrict__ B,
+                                          int S, int i0, int j0, double acc[4][4][2],
+                                          NewtonSmem& sm) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wm = warp >> 1, wn = warp & 1;
+  auto load = [&](int stage, int k0) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int c = tid + r * kNewtonThreads;          // 512 16-byte chunks per operand
+      const int ar = c >> 3, ac = (c & 7) * 2;         // A: 64 rows x 8 chunks
+      cp_async16(&sm.As[stage][ar][ac], A + (size_t)(i0 + ar) * S + k0 + ac);
+      const int br = c >> 5, bc = (c & 31) * 2;        // B: 16 rows x 32 chunks
+      cp_async16(&sm.Bs[stage][br][bc], B + (size_t)(k0 + br) * S + j0 + bc);
+    }
+    cp_async_commit();
+  };
+  const int nk = S / kBK;
+  load(0, 0);
+  for (int kt = 0; kt < nk; ++kt) {
+    if (kt + 1 < nk) {
+      load((kt + 1) & 1, (kt + 1) * kBK);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int st = kt & 1;
+#pragma unroll
+    for (int kk = 0; kk < kBK; kk += 4) {
+      double a[4], b[4];
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi) a[mi] = sm.As[st][wm * 32 + mi * 8 + g][kk + t];
+#pragma unroll
+      for (int ni = 0; ni < 4; ++ni) b[ni] = sm.Bs[st][kk + t][wn * 32 + ni * 8 + g];
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) dmma884(acc[mi][ni][0], acc[mi][ni][1], a[mi], b[ni]);
+    }
+    __syncthreads();
+  }
+}
+
+// Store the tile to C at (i0, j0) and, off the diagonal, its transpose at (j0, i0).
+__device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0, int j0,
+                                          const double acc[4][4][2]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wm = warp >> 1, wn = warp & 1;
+#pragma unroll
+  for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni) {
+      const int r = i0 + wm * 32 + mi * 8 + g;
+      const int c = j0 + wn * 32 + ni * 8 + 2 * t;
+      *reinterpret_cast<double2*>(C + (size_t)r * S + c) = make_double2(acc[mi][ni][0], acc[mi][ni][1]);
+      if (i0 != j0) {
+        C[(size_t)c * S + r] = acc[mi][ni][0];
+        C[(size_t)(c + 1) * S + r] = acc[mi][ni][1];
+      }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Set-up: the eigenvalue bound, X0, M0, T0 and the first residual.
+// ---------------------------------------------------------------------------
+// One CTA per matrix: c^p = min(||A + eps I||_F, ||A + eps I||_inf) over the
+// valid corner.  Both bound the largest eigenvalue of a symmetric matrix.
+__global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restrict__ A,
+                                                           int64_t a_stride, int lda,
+                                                           const NewtonMat* __restrict__ mats,
+                                                           float eps, double* __restrict__ cinv,
+                                                           double* __restrict__ cpow) {
+  __shared__ double red[8];
+  const NewtonMat mt = mats[blockIdx.x];
+  const float* a = A + (size_t)mt.slot * a_stride;
+  const int n = mt.size;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double fro = 0.0, rowmax = 0.0;
+  for (int r = warp; r < n; r += 8) {
+    double rs = 0.0;
+    for (int c = lane; c < n; c += 32) {
+      double v = (double)a[(size_t)r * lda + c];
+      if (r == c) v += (double)eps;
+      rs += fabs(v);
+      fro += v * v;
+    }
+    rs = warp_sum(rs);
+    rowmax = fmax(rowmax, rs);
+  }
+  fro = block_sum(fro, red);
+  rowmax = block_max(rowmax, red);
+  if (threadIdx.x == 0) {
+    double cp = fmin(sqrt(fro), rowmax);
+    if (!(cp > 0.0) || !(cp <= DBL_MAX)) cp = (cp > 0.0) ? cp : 1.0;  // NaN/Inf/0 caught later
+    cpow[blockIdx.x] = cp;
+    cinv[blockIdx.x] = pow(cp, -1.0 / mt.p);
+  }
+}
+
+// grid: x = row of the S x S slot, y = matrix.  Writes X0, M0, T0 into the
+// parity-0 buffers and folds max|M0 - I| into the residual.
+__global__ void __launch_bounds__(256) newton_init_kernel(const float* __restrict__ A,
+                                                          int64_t a_stride, int lda,
+                                                          const NewtonMat* __restrict__ mats,
+                                                          int S, float eps, NewtonWork w,
+                                                          const double* __restrict__ cpow) {
+  __shared__ double red[8];
+  const int m = blockIdx.y;
+  const NewtonMat mt = mats[m];
+  const float* a = A + (size_t)mt.slot * a_stride;
+  const int r = blockIdx.x;
+  const size_t off = (size_t)m * S * S + (size_t)r * S;
+  const double inv_cp = 1.0 / cpow[m];
+  const double ci = w.cinv[m];
+  const double pinv = 1.0 / mt.p;
+  double dev = 0.0;
+  for (int c = threadIdx.x; c < S; c += blockDim.x) {
+    double v;
+    if (r < mt.size && c < mt.size) {
+      v = (double)a[(size_t)r * lda + c];
+      if (r == c) v += (double)eps;
+      v *= inv_cp;
+    } else {
+      v = (r == c) ? 1.0 : 0.0;
+    }
+    const double d = (r == c) ? 1.0 : 0.0;
+    w.M[0][off + c] = v;
+    w.T[off + c] = ((mt.p + 1) * d - v) * pinv;
+    w.X[0][off + c] = (r == c) ? ci : 0.0;
+    double e = fabs(v - d);
+    if (!(e <= DBL_MAX)) e = INFINITY;
+    dev = fmax(dev, e);
+  }
+  dev = block_max(dev, red);
+  if (threadIdx.x == 0) atomicMax(&w.resid[m], dbl_bits(dev));
+}
+
+// ---------------------------------------------------------------------------
+// One Newton step, three launches:
+//   job 0: X_next = X T      job 1: T2 = T T            (launch A)
+//   T4 = T2 T2 (p = 4 only)                              (launch B)
+//   M_next = T^p M, residual, T <- ((p+1) I - M_next)/p  (launch C)
+// grid: x = upper-triangular tile, y = matrix, z = job.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kNewtonThreads) newton_step_a_kernel(
+    const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
+  __shared__ NewtonSmem sm;
+  const int m = blockIdx.y;
+  if (w.state[m] != kRunning) return;
+  const int T = S / kTile;
+  int ti, tj;
+  tri_tile(blockIdx.x, T, ti, tj);
+  const size_t base = (size_t)m * S * S;
+  const double* Tm = w.T + base;
+  const double* A = blockIdx.z == 0 ? w.X[it & 1] + base : Tm;
+  double* C = blockIdx.z == 0 ? w.X[(it + 1) & 1] + base : w.T2 + base;
+  double acc[4][4][2] = {};
+  dmma_tile(A, Tm, S, ti * kTile, tj * kTile, acc, sm);
+  store_sym(C, S, ti * kTile, tj * kTile, acc);
+}
+
+__global__ void __launch_bounds__(kNewtonThreads) newton_step_b_kernel(
+    const NewtonMat* __restrict__ mats, int S, NewtonWork w) {
+  __shared__ NewtonSmem sm;
+  const int m = blockIdx.y;
+  if (w.state[m] != kRunning || mats[m].p != 4) return;
+  const int T = S / kTile;
+  int ti, tj;
+  tri_tile(blockIdx.x, T, ti, tj);
+  const size_t base = (size_t)m * S * S;
+  double acc[4][4][2] = {};
+  dmma_tile(w.T2 + base, w.T2 + base, S, ti * kTile, tj * kTile, acc, sm);
+  store_sym(w.T4 + base, S, ti * kTile, tj * kTile, acc);
+}
+
+__global__ void __launch_bounds__(kNewtonThreads) newton_step_c_kernel(
+    const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
+  __shared__ NewtonSmem sm;
+  __shared__ double red[kNewtonThreads / 32];
+  const int m = blockIdx.y;
+  if (w.state[m] != kRunning) return;
+  const int p = mats[m].p;
+  const int T = S / kTile;
+  int ti, tj;
+  tri_tile(blockIdx.x, T, ti, tj);
+  const size_t base = (size_t)m * S * S;
+  const double* Tp = (p == 4 ? w.T4 : w.T2) + base;
+  double acc[4][4][2] = {};
+  const int i0 = ti * kTile, j0 = tj * kTile;
+  dmma_tile(Tp, w.M[it & 1] + base, S, i0, j0, acc, sm);
+  store_sym(w.M[(it + 1) & 1] + base, S, i0, j0, acc);
+  // residual and the next T from the same accumulators
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int wm = warp >> 1, wn = warp & 1;
+  const double pinv = 1.0 / p;
+  double dev = 0.0;
+#pragma unroll
+  for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = i0 + wm * 32 + mi * 8 + g;
+        const int c = j0 + wn * 32 + ni * 8 + 2 * t + e;
+        const double d = (r == c) ? 1.0 : 0.0;
+        double x = fabs(acc[mi][ni][e] - d);
+        if (!(x <= DBL_MAX)) x = INFINITY;
+        dev = fmax(dev, x);
+        acc[mi][ni][e] = ((p + 1) * d - acc[mi][ni][e]) * pinv;
+      }
+  store_sym(w.T + base, S, i0, j0, acc);
+  dev = block_max(dev, red);
+  if (threadIdx.x == 0) atomicMax(&w.resid[m], dbl_bits(dev));
+}
+
+// Convergence test of M_k for every matrix (k = iterations done), in the
+// same order as the oracle: non-finite, tolerance, cap, 5 non-decreasing.
+__global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, NewtonWork w) {
+  int alive = 0;
+  for (int m = threadIdx.x; m < nm; m += blockDim.x) {
+    if (w.state[m] != kRunning) continue;
+    const double r = __longlong_as_double(static_cast<long long>(w.resid[m]));
+    w.resid[m] = 0ull;
+    w.iters[m] = k;
+    int st = kRunning;
+    if (!(r <= DBL_MAX)) {
+      st = kFailed;
+    } else if (r <= tol) {
+      st = kConverged;
+    } else if (k >= max_iters) {
+      st = kFailed;
+    } else {
+      const int wo = (r >= w.prev[m]) ? w.worse[m] + 1 : 0;
+      w.worse[m] = wo;
+      w.prev[m] = r;
+      if (wo >= 5) st = kFailed;
+    }
+    w.state[m] = st;
+    alive += (st == kRunning);
+  }
+  // number of threads still holding a running matrix: zero iff none runs
+  alive = __syncthreads_count(alive);
+  if (threadIdx.x == 0) w.count[k & 1] = alive;
+}
+
+__global__ void newton_reset_kernel(int nm, NewtonWork w) {
+  for (int m = threadIdx.x; m < nm; m += blockDim.x) {
+    w.state[m] = kRunning;
+    w.resid[m] = 0ull;
+    w.prev[m] = INFINITY;
+    w.worse[m] = 0;
+    w.iters[m] = 0;
+  }
+}
+
+// grid: x = row, y = matrix.  Converged: X (float32) from the final buffer.
+// Failed: keep the old root if there is one, else write c^{-1} I.
+__global__ void __launch_bounds__(256) newton_finalize_kernel(
+    float* __restrict__ X, int64_t x_stride, int ldx, const NewtonMat* __restrict__ mats, int S,
+    NewtonWork w, int* __restrict__ has_root, int32_t* __restrict__ iters_out) {
+  const int m = blockIdx.y;
+  const NewtonMat mt = mats[m];
+  const int st = w.state[m];
+  const int r = blockIdx.x;
+  if (r >= ldx) return;
+  const bool ok = (st == kConverged);
+  if (!ok && has_root && has_root[mt.slot]) return;
+  float* x = X + (size_t)mt.slot * x_stride + (size_t)r * ldx;
+  const double* src = w.X[w.iters[m] & 1] + (size_t)m * S * S + (size_t)r * S;
+  const double ci = w.cinv[m];
+  for (int c = threadIdx.x; c < ldx; c += blockDim.x) {
+    double v = 0.0;
+    if (r < mt.size && c < mt.size) v = ok ? src[c] : (r == c ? ci : 0.0);
+    x[c] = (float)v;
+  }
+  __syncthreads();
+  if (r == 0 && threadIdx.x == 0) {
+    if (ok && has_root) has_root[mt.slot] = 1;
+    if (iters_out) iters_out[mt.slot] = ok ? w.iters[m] : -1 - w.iters[m];
+  }
+}
+
+}  // namespace
+
+void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s) {
+  newton_reset_kernel<<<1, 1024, 0, s>>>(nm, w);
+}
+
+// c^p goes to the first nm doubles of T2, which no step reads before step A
+// overwrites it.
+void launch_newton_bound(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
+                         float eps, NewtonWork w, cudaStream_t s) {
+  newton_bound_kernel<<<nm, 256, 0, s>>>(A, a_stride, lda, mats, eps, w.cinv, w.T2);
+}
+
+void launch_newton_init(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
+                        int S, float eps, NewtonWork w, cudaStream_t s) {
+  newton_init_kernel<<<dim3(S, nm), 256, 0, s>>>(A, a_stride, lda, mats, S, eps, w, w.T2);
+}
+
+static int num_tri(int S) {
+  const int T = S / kTile;
+  return T * (T + 1) / 2;
+}
+
+void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s) {
+  newton_step_a_kernel<<<dim3(num_tri(S), nm, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+}
+
+void launch_newton_step_b(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {
+  newton_step_b_kernel<<<dim3(num_tri(S), nm), kNewtonThreads, 0, s>>>(mats, S, w);
+}
+
+void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s) {
+  newton_step_c_kernel<<<dim3(num_tri(S), nm), kNewtonThreads, 0, s>>>(mats, S, it, w);
+}
+
+void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s) {
+  newton_check_kernel<<<1, 1024, 0, s>>>(nm, k, tol, max_iters, w);
+}
+
+void launch_newton_finalize(float* X, int64_t x_stride, int ldx, const NewtonMat* mats, int nm,
+                            int S, NewtonWork w, int* has_root, int32_t* iters_out,
+                            cudaStream_t s) {
+  newton_finalize_kernel<<<dim3(ldx, nm), 256, 0, s>>>(X, x_stride, ldx, mats, S, w, has_root,
+                                                       iters_out);
+}
+
+}  // namespace shampoo

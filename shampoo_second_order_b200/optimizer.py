@@ -1,0 +1,114 @@
+"""Torch-facing handle over the C-ABI: holds one library context and passes
+tensor data pointers and the current CUDA stream to it.  All arithmetic runs
+in the CUDA library."""
+from __future__ import annotations
+
+import numpy as np
+
+from . import _lib as L
+
+
+class Shampoo:
+    """One optimizer state for a fixed list of parameter shapes.
+
+    shapes: (rows, cols) for 2-D parameters, (n,) for 1-D ones.  Gradients
+    are float32 or bfloat16 CUDA tensors (grad_dtype "f32" / "bf16"),
+    parameters float32 CUDA tensors, all contiguous.
+    """
+
+    def __init__(self, shapes, block_size, beta2, eps, p=4, graft=L.GRAFT_ADAGRAD, momentum=0.0,
+                 grad_dtype="f32", stream=None):
+        import torch
+        self.shapes = [tuple(s) for s in shapes]
+        self.block_size = int(block_size)
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        self.stream = stream
+        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        dt = L.BF16 if grad_dtype == "bf16" else L.F32
+        self.ctx = L.shampoo_create(self.shapes, block_size, beta2, eps, p, graft, momentum, dt, handle)
+
+    def _check_tensors(self, ts, what):
+        if len(ts) != len(self.shapes):
+            raise ValueError(f"expected {len(self.shapes)} {what}, got {len(ts)}")
+        for t, s in zip(ts, self.shapes):
+            if not (t.is_cuda and t.is_contiguous()) or t.numel() != int(np.prod(s)):
+                raise ValueError(f"{what} must be contiguous CUDA tensors of the given shapes")
+
+    def update_stats(self, grads):
+        self._check_tensors(grads, "grads")
+        L.shampoo_update_stats(self.ctx, grads)
+
+    def compute_roots(self):
+        """Returns True when every root converged."""
+        return L.shampoo_compute_roots(self.ctx) == L.OK
+
+    def apply(self, params, grads, lr):
+        self._check_tensors(params, "params")
+        self._check_tensors(grads, "grads")
+        L.shampoo_apply(self.ctx, params, grads, lr)
+
+    def step(self, params, grads, lr, compute_roots):
+        self.update_stats(grads)
+        if compute_roots:
+            self.compute_roots()
+        self.apply(params, grads, lr)
+
+    def root_status(self):
+        return L.shampoo_root_status(self.ctx)
+
+    def nonfinite_status(self):
+        return L.shampoo_nonfinite_status(self.ctx)
+
+    def set_root_options(self, tol, max_iters):
+        L.shampoo_set_root_options(self.ctx, tol, max_iters)
+
+    def root_iterations(self):
+        return L.shampoo_root_iterations(self.ctx)
+
+    def profile_enable(self, on=True):
+        L.shampoo_profile_enable(self.ctx, on)
+
+    def profile_read(self):
+        return L.shampoo_profile_read(self.ctx)
+
+    def num_matrices(self):
+        return L.shampoo_num_matrices(self.ctx)
+
+    def matrix_info(self, index):
+        return L.shampoo_matrix_info(self.ctx, index)
+
+    def read_matrix(self, which, index):
+        """The valid corner of statistic `index` (which=0) or its root
+        (which=1) as a float32 numpy array."""
+        b = self.block_size
+        out = np.zeros((b, b), dtype=np.float32)
+        L.shampoo_read_matrix(self.ctx, which, index, out.ctypes.data)
+        size, _ = self.matrix_info(index)
+        return out[:size, :size].copy(), out
+
+    def close(self):
+        if self.ctx is not None:
+            L.shampoo_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def batched_inverse_root(A, p, eps, tol=1e-6, max_iters=100, stream=None):
+    """X = (A + eps I)^{-1/p} for a float32 CUDA tensor A [batch, n, n].
+    Returns (X, iters) with iters an int32 CUDA tensor (negative = gave up)."""
+    import torch
+    assert A.is_cuda and A.dtype == torch.float32 and A.dim() == 3 and A.is_contiguous()
+    batch, n, _ = A.shape
+    X = torch.empty_like(A)
+    iters = torch.empty(batch, dtype=torch.int32, device=A.device)
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    L.shampoo_batched_inverse_root(A.data_ptr(), X.data_ptr(), batch, n, p, eps, tol, max_iters,
+                                   iters.data_ptr(), stream.cuda_stream)
+    return X, iters

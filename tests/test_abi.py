@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point
+include/shampoo.h declares, and rejects bad arguments on the host with
+SHAMPOO_EINVAL before touching the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from shampoo_second_order_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(shampoo_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(L.LIB_PATH):
+        import __graft_entry__
+        __graft_entry__.build()
+    return L.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "shampoo_create" in names and "shampoo_batched_inverse_root" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(L.SIGNATURES), set(names) - set(L.SIGNATURES)
+
+
+def test_version(lib):
+    assert re.match(r"^\d+\.\d+\.\d+$", L.shampoo_version())
+
+
+@pytest.mark.parametrize("kw,msg", [
+    (dict(block_size=100), "block_size"),
+    (dict(block_size=32), "block_size"),
+    (dict(block_size=2048), "block_size"),
+    (dict(beta2=0.0), "beta2"),
+    (dict(beta2=1.5), "beta2"),
+    (dict(epsilon=0.0), "epsilon"),
+    (dict(p=3), "p must"),
+    (dict(graft=7), "graft"),
+    (dict(momentum=1.0), "momentum"),
+    (dict(grad_dtype=5), "dtype"),
+])
+def test_create_rejects_bad_options(lib, kw, msg):
+    args = dict(shapes=[(64, 32)], block_size=64, beta2=1.0, epsilon=1e-6, p=4, graft=1,
+                momentum=0.0, grad_dtype=0)
+    args.update(kw)
+    with pytest.raises(L.ShampooError) as e:
+        L.shampoo_create(args["shapes"], args["block_size"], args["beta2"], args["epsilon"],
+                         args["p"], args["graft"], args["momentum"], args["grad_dtype"])
+    assert e.value.status == L.EINVAL and msg in str(e.value)
+
+
+def test_create_rejects_bad_shapes(lib):
+    ctx = C.c_void_p()
+    dims = (C.c_int64 * 2)(0, 5)
+    assert lib.shampoo_create(C.byref(ctx), 1, dims, None, 64, 1.0, 1e-6, 4, 1, 0.0, 0, None) == L.EINVAL
+    dims = (C.c_int64 * 2)(3, 5)
+    nd = (C.c_int32 * 1)(1)          # 1-D must be given as (1, n)
+    assert lib.shampoo_create(C.byref(ctx), 1, dims, nd, 64, 1.0, 1e-6, 4, 1, 0.0, 0, None) == L.EINVAL
+    assert lib.shampoo_create(C.byref(ctx), 0, dims, None, 64, 1.0, 1e-6, 4, 1, 0.0, 0, None) == L.EINVAL
+    assert lib.shampoo_create(None, 1, dims, None, 64, 1.0, 1e-6, 4, 1, 0.0, 0, None) == L.EINVAL
+    assert not ctx.value
+
+
+def test_null_context_calls(lib):
+    assert lib.shampoo_update_stats(None, None) == L.EINVAL
+    assert lib.shampoo_compute_roots(None) == L.EINVAL
+    assert lib.shampoo_apply(None, None, None, 0.1) == L.EINVAL
+    assert lib.shampoo_num_matrices(None) == 0
+    lib.shampoo_destroy(None)
+
+
+@pytest.mark.parametrize("args", [
+    (0, 0, 1, 64, 4, 1e-6, 1e-6, 100),        # null pointers
+    (8, 8, 0, 64, 4, 1e-6, 1e-6, 100),        # batch 0
+    (8, 8, 1, 2048, 4, 1e-6, 1e-6, 100),      # n too large
+    (8, 8, 1, 64, 3, 1e-6, 1e-6, 100),        # p
+    (8, 8, 1, 64, 4, 0.0, 1e-6, 100),         # eps
+    (8, 8, 1, 64, 4, 1e-6, 1e-6, 0),          # max_iters
+])
+def test_batched_root_rejects_bad_arguments(lib, args):
+    a, x, batch, n, p, eps, tol, mi = args
+    st = lib.shampoo_batched_inverse_root(C.c_void_p(a), C.c_void_p(x), batch, n, p, eps, tol, mi,
+                                          None, None)
+    assert st == L.EINVAL
+
+
+def test_package_import_does_not_load_library():
+    import importlib
+    import shampoo_second_order_b200 as pkg
+    importlib.reload(pkg)
+    from shampoo_second_order_b200 import workloads  # noqa: F401
+    assert hasattr(pkg, "lib")

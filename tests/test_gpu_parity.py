@@ -1,0 +1,249 @@
+"""Parity of the CUDA path with the fp64 oracle, through the C-ABI.
+
+Tolerances (relative Frobenius error per object):
+  statistics L, R, S              <= 1e-5
+  roots, condition number <= 1e6  <= 1e-3
+  per block: W_new and the step dW = W_new - W_old   <= 1e-3
+Both sides take the same seeded inputs from the workloads module; the oracle
+never sees a value the CUDA path produced except where a test compares.
+"""
+import numpy as np
+import pytest
+
+from oracle import ShampooOracle, block_partition, inverse_root, vector_segments
+from shampoo_second_order_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+STATS_TOL = 1e-5
+ROOT_TOL = 1e-3
+STEP_TOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from shampoo_second_order_b200 import _lib
+    _lib.lib()   # fails loudly if the library is missing
+    yield
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def to_dev(x, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def pieces(shape, b):
+    if len(shape) == 2:
+        return [(slice(r0, r0 + m), slice(c0, c0 + n)) for (r0, c0, m, n) in block_partition(*shape, b)]
+    return [(slice(s0, s0 + ln),) for (s0, ln) in vector_segments(shape[0], b)]
+
+
+def run_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, interval, seed, gstd,
+             check_every=True, check_state=True):
+    from shampoo_second_order_b200 import Shampoo
+    o = ShampooOracle(shapes, b, beta2, eps, 4, graft, mu)
+    opt = Shampoo(shapes, b, beta2, eps, 4, graft, mu, gdtype)
+    W0 = wl.make_params(shapes, seed)
+    Wo = [w.astype(np.float64) for w in W0]
+    Wd = [torch.from_numpy(w).cuda() for w in W0]
+    worst = {"stats": 0.0, "roots": 0.0, "dW": 0.0, "W": 0.0}
+    for t in range(steps):
+        g = wl.make_grads(shapes, seed, t, gstd, gdtype)
+        gd = [to_dev(x, gdtype) for x in g]
+        roots = (t % interval == 0)
+        prev_d = [w.cpu().numpy().astype(np.float64) for w in Wd]
+        prev_o = Wo
+        Wo = o.step(Wo, g, lr, roots)
+        opt.step(Wd, gd, lr, roots)
+        torch.cuda.synchronize()
+        if not (check_every or t == steps - 1):
+            continue
+        if check_state and (roots or t == steps - 1):
+            mats = o.matrices()
+            ro = o.root_matrices()
+            for k in range(opt.num_matrices()):
+                S, _ = opt.read_matrix(0, k)
+                worst["stats"] = max(worst["stats"], rel(S, mats[k][0]))
+                X, _ = opt.read_matrix(1, k)
+                worst["roots"] = max(worst["roots"], rel(X, ro[k]))
+        for i, s in enumerate(shapes):
+            wd = Wd[i].cpu().numpy().astype(np.float64)
+            for sl in pieces(s, b):
+                worst["dW"] = max(worst["dW"], rel((wd - prev_d[i])[sl], (Wo[i] - prev_o[i])[sl]))
+                worst["W"] = max(worst["W"], rel(wd[sl], Wo[i][sl]))
+    opt.close()
+    return worst
+
+
+def assert_worst(w):
+    assert w["stats"] <= STATS_TOL, w
+    assert w["roots"] <= ROOT_TOL, w
+    assert w["dW"] <= STEP_TOL, w
+    assert w["W"] <= STEP_TOL, w
+
+
+# --------------------------------------------------------------------------
+# whole steps on small cases (several tiles, ragged tails, both grad dtypes)
+# --------------------------------------------------------------------------
+def test_single_64x32_ten_steps():
+    c = wl.CONFIGS["single_64x32"]
+    w = run_pair(c["shapes"], c["block_size"], c["beta2"], c["eps"], c["graft"], c["momentum"],
+                 c["lr"], c["grad_dtype"], c["steps"], c["root_interval"], c["seed"], c["grad_std"])
+    assert_worst(w)
+
+
+@pytest.mark.parametrize("gdtype", ["f32", "bf16"])
+@pytest.mark.parametrize("graft,mu", [(1, 0.0), (0, 0.0), (1, 0.9)])
+def test_ragged_mixed_set(gdtype, graft, mu):
+    shapes = [(200, 130), (64, 64), (19, 200), (130,), (64,), (1, 77)]
+    w = run_pair(shapes, 64, 0.99, 1e-6, graft, mu, 0.1, gdtype, steps=6, interval=3, seed=7,
+                 gstd=1e-2)
+    assert_worst(w)
+
+
+def test_block_128_many_tiles():
+    shapes = [(300, 257), (128, 384), (500,)]
+    w = run_pair(shapes, 128, 0.999, 1e-6, 1, 0.0, 0.1, "f32", steps=4, interval=2, seed=8, gstd=1e-3)
+    assert_worst(w)
+
+
+def test_transformer_layer_b512_full_size():
+    """The Transformer-layer set at full size in the bench's launch
+    configuration: 21 steps, roots at steps 1 and 21."""
+    c = wl.CONFIGS["transformer_layer_b512"]
+    w = run_pair(c["shapes"], c["block_size"], c["beta2"], c["eps"], c["graft"], c["momentum"],
+                 c["lr"], c["grad_dtype"], 21, c["root_interval"], c["seed"], c["grad_std"],
+                 check_every=False)
+    assert_worst(w)
+
+
+# --------------------------------------------------------------------------
+# the batched inverse-root kernel on its own
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [64, 100, 192, 512])
+@pytest.mark.parametrize("p", [2, 4])
+def test_batched_root_vs_oracle(n, p):
+    from shampoo_second_order_b200 import batched_inverse_root
+    A, _ = wl.spd_batch(6, n, seed=n + p, log10_kappa=(2.0, 6.0))
+    A32 = A.astype(np.float32)
+    X, iters = batched_inverse_root(torch.from_numpy(A32).cuda(), p, 1e-6)
+    X = X.cpu().numpy()
+    iters = iters.cpu().numpy()
+    assert (iters > 0).all(), iters
+    for i in range(6):
+        ref = inverse_root(A32[i].astype(np.float64), 1e-6, p)
+        assert rel(X[i], ref) <= ROOT_TOL, (i, rel(X[i], ref))
+
+
+def test_batched_root_kappa_sweep_full_size():
+    """256 SPD 512 x 512 matrices with condition numbers 1e2..1e8; every
+    matrix with kappa <= 1e6 within 1e-3, sampled against the oracle."""
+    from shampoo_second_order_b200 import batched_inverse_root
+    c = wl.ROOTS_CONFIG
+    A, lam = wl.spd_batch(c["batch"], c["n"], c["seed"], c["log10_kappa"])
+    A32 = A.astype(np.float32)
+    dA = torch.from_numpy(A32).cuda()
+    for p in c["ps"]:
+        X, iters = batched_inverse_root(dA, p, c["eps"], c["tol"])
+        X = X.cpu().numpy()
+        iters = iters.cpu().numpy()
+        kappa = lam.max(1) / lam.min(1)
+        for i in list(range(0, c["batch"], 16)) + [c["batch"] - 1]:
+            ref = inverse_root(A32[i].astype(np.float64), c["eps"], p)
+            if kappa[i] <= 1e6:
+                assert iters[i] > 0
+                assert rel(X[i], ref) <= ROOT_TOL, (p, i, kappa[i], rel(X[i], ref))
+
+
+# --------------------------------------------------------------------------
+# edge cases and error conventions
+# --------------------------------------------------------------------------
+def test_zero_gradient_leaves_weight():
+    from shampoo_second_order_b200 import Shampoo
+    shapes = [(70, 70), (33,)]
+    opt = Shampoo(shapes, 64, 0.9, 1e-6)
+    W = [torch.randn(s, device="cuda") for s in shapes]
+    W0 = [w.clone() for w in W]
+    g = [torch.zeros(s, device="cuda") for s in shapes]
+    opt.step(W, g, 0.1, True)
+    torch.cuda.synchronize()
+    for a, b in zip(W, W0):
+        assert torch.equal(a, b)
+    opt.close()
+
+
+def test_nonfinite_gradient_skips_parameter():
+    from shampoo_second_order_b200 import Shampoo
+    shapes = [(64, 40), (50, 64)]
+    opt = Shampoo(shapes, 64, 0.9, 1e-6)
+    W = [torch.randn(s, device="cuda") for s in shapes]
+    g = [torch.randn(s, device="cuda") for s in shapes]
+    opt.step(W, g, 0.1, True)
+    W1 = [w.clone() for w in W]
+    L_before, _ = opt.read_matrix(0, 0)
+    g2 = [torch.randn(s, device="cuda") for s in shapes]
+    g2[0][3, 5] = float("nan")
+    opt.step(W, g2, 0.1, False)
+    torch.cuda.synchronize()
+    assert opt.nonfinite_status() == 1
+    assert torch.equal(W[0], W1[0])
+    assert not torch.equal(W[1], W1[1])
+    L_after, _ = opt.read_matrix(0, 0)
+    assert np.array_equal(L_before, L_after)
+    opt.close()
+
+
+def test_apply_before_roots_is_state_error():
+    from shampoo_second_order_b200 import Shampoo, _lib
+    opt = Shampoo([(64, 64)], 64, 1.0, 1e-6)
+    W = [torch.zeros(64, 64, device="cuda")]
+    g = [torch.randn(64, 64, device="cuda")]
+    opt.update_stats(g)
+    with pytest.raises(_lib.ShampooError) as e:
+        opt.apply(W, g, 0.1)
+    assert e.value.status == _lib.ESTATE
+    opt.close()
+
+
+def test_iteration_cap_reports_not_converged_and_falls_back():
+    from shampoo_second_order_b200 import Shampoo
+    opt = Shampoo([(64, 32)], 64, 1.0, 1e-6)
+    opt.set_root_options(1e-6, 2)
+    g = [torch.randn(64, 32, device="cuda")]
+    opt.update_stats(g)
+    assert opt.compute_roots() is False
+    nf, it = opt.root_status()
+    assert nf == 2 and it == 2
+    # never had a root: c^{-1} I with c^p = min(||A+eps I||_F, ||A+eps I||_inf)
+    L, _ = opt.read_matrix(0, 0)
+    A = (g[0].double() @ g[0].double().T).cpu().numpy() + 1e-6 * np.eye(64)
+    cp = min(np.linalg.norm(A), np.abs(A).sum(1).max())
+    X, _ = opt.read_matrix(1, 0)
+    assert np.allclose(X, cp ** -0.25 * np.eye(64), rtol=1e-5)
+    # with the cap lifted they converge and replace the fallback
+    opt.set_root_options(1e-6, 100)
+    assert opt.compute_roots() is True
+    X2, _ = opt.read_matrix(1, 0)
+    assert rel(X2, inverse_root(opt.read_matrix(0, 0)[0].astype(np.float64), 1e-6, 4)) < ROOT_TOL
+    opt.close()
+
+
+def test_nan_statistic_fails_root_and_keeps_previous():
+    from shampoo_second_order_b200 import batched_inverse_root
+    A = np.stack([np.eye(64, dtype=np.float32) * 2, np.eye(64, dtype=np.float32)])
+    A[1, 3, 3] = np.nan
+    X, iters = batched_inverse_root(torch.from_numpy(A).cuda(), 4, 1e-6)
+    iters = iters.cpu().numpy()
+    assert iters[0] >= 0 and iters[1] < 0
+    assert np.allclose(X[0].cpu().numpy(), (2 + 1e-6) ** -0.25 * np.eye(64), rtol=1e-6)
