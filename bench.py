@@ -143,13 +143,21 @@ class ClockSampler:
                     rows.append(parts)
         os.unlink(self.f.name)
         if not rows:
-            return None
+            return {"error": "no nvidia-smi samples"}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
 
 
 def fp64_peak_tflops(torch, dev):
@@ -286,6 +294,57 @@ def reference_arm(args, cfg, rank, world):
 
 
 # ---------------------------------------------------------------------------
+# the batched inverse-root kernel on its own (256 SPD 512 x 512, p = 4 and 2)
+# ---------------------------------------------------------------------------
+def roots_bench(args):
+    import torch
+    from shampoo_second_order_b200 import batched_inverse_root
+    c = wl.ROOTS_CONFIG
+    batch = args.batch or c["batch"]
+    A, lam = wl.spd_batch(batch, c["n"], c["seed"], c["log10_kappa"])
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        dA = torch.from_numpy(A.astype(np.float32)).to(dev)
+        flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+        fp64_peak = fp64_peak_tflops(torch, dev)
+    n = c["n"]
+    flops = 0
+    ev = []
+    for j in range(args.warmup + args.steps):
+        timed = j >= args.warmup
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            its = []
+            for p in c["ps"]:
+                X, it = batched_inverse_root(dA, p, c["eps"], c["tol"], stream=stream)
+                its.append((p, it))
+            e.record(stream)
+        stream.synchronize()
+        if timed:
+            ev.append((s, e))
+            for p, it in its:
+                k = it.cpu().numpy()
+                k = np.where(k >= 0, k, -1 - k)
+                flops += int(k.sum()) * (4 if p == 4 else 3) * n * n * (n + 1)
+    ms = sum(s.elapsed_time(e) for s, e in ev)
+    val = flops / (ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "batched_roots_512", "batch": batch, "n": n, "p": list(c["ps"]),
+                       "tol": c["tol"], "l2": "flushed between steps (256 MiB write)"},
+            "roofline": {"kernel": "newton (all launches of one call)", "bound": "tensor",
+                         "achieved": round(val, 3), "peak": round(fp64_peak, 2), "unit": "TFLOP/s",
+                         "frac": round(val / fp64_peak, 4), "traffic": None,
+                         "peak_source": "cuBLAS DGEMM measured in this run"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # the CUDA arm
 # ---------------------------------------------------------------------------
 def main():
@@ -294,10 +353,15 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--config", default="transformer_layer_b512", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--config", default="transformer_layer_b512",
+                    choices=sorted(wl.CONFIGS) + ["batched_roots_512"])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="batched_roots_512 only: number of matrices (default 256)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
+    if args.config == "batched_roots_512":
+        return roots_bench(args)
     cfg = wl.CONFIGS[args.config]
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -361,11 +425,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    uuid = None
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
+    uuid = gpu_uuid(torch, dev)
     clocks = ClockSampler(uuid)
     opt.profile_enable(True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

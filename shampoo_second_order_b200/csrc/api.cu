@@ -131,6 +131,7 @@ struct shampoo_ctx {
   int* flags = nullptr;
   int* has_root = nullptr;
   NewtonWork nw{};
+  NewtonMat* d_retry = nullptr;
   int newton_chunk = 0;
   int* h_count = nullptr;   // pinned [2]
   cudaEvent_t ev[2] = {nullptr, nullptr};
@@ -191,6 +192,7 @@ cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
   for (auto b : bufs)
     if ((e = dalloc(ctx, b, mat)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.cinv, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.ridge, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.resid, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.prev, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.worse, chunk)) != cudaSuccess) return e;
@@ -203,52 +205,80 @@ cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
 // Run the Newton iteration over mats[0..nm) (device array dm) in chunks of
 // `chunk` matrices.  A/X are float32 slot arrays.  Returns the number of
 // matrices that gave up and the largest iteration count through outs.
+// Run the Newton iteration over the matrices hm (device copy dm) in chunks of
+// `chunk`.  A matrix whose iteration diverges (rounding left A + eps I
+// indefinite) is run again with the ridge raised, up to kAttempts times.
+// Reports the number of matrices that gave up, the largest iteration count
+// and, per matrix slot, the iterations (-1-k when it gave up at k).
+constexpr int kAttempts = 4;
+
 shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<NewtonMat>& hm,
-                          const NewtonMat* dm, const float* A, int64_t a_stride, int lda, float* X,
-                          int64_t x_stride, int ldx, int S, float eps, double tol, int max_iters,
-                          int chunk, NewtonWork& w, int* has_root, int32_t* iters_out, int* h_count,
-                          cudaEvent_t* ev, cudaStream_t st, int* n_failed, int* max_it,
-                          std::vector<int32_t>* per_matrix) {
+                          const NewtonMat* dm, NewtonMat* d_retry, const float* A,
+                          int64_t a_stride, int lda, float* X, int64_t x_stride, int ldx, int S,
+                          float eps, double tol, int max_iters, int chunk, NewtonWork& w,
+                          int* has_root, int32_t* iters_out, int* h_count, cudaEvent_t* ev,
+                          cudaStream_t st, int* n_failed, int* max_it,
+                          std::vector<int32_t>* per_slot) {
   *n_failed = 0;
   *max_it = 0;
   const int nm_all = (int)hm.size();
-  if (per_matrix) per_matrix->assign(nm_all, 0);
+  int max_slot = 0;
+  for (const auto& m : hm) max_slot = std::max(max_slot, m.slot + 1);
+  if (per_slot) per_slot->assign(max_slot, 0);
   std::vector<int> hstate(chunk), hiters(chunk);
   for (int c0 = 0; c0 < nm_all; c0 += chunk) {
-    const int nm = std::min(chunk, nm_all - c0);
+    std::vector<NewtonMat> list(hm.begin() + c0, hm.begin() + std::min(nm_all, c0 + chunk));
     const NewtonMat* d = dm + c0;
-    int has_p4 = 0;
-    for (int i = 0; i < nm; ++i) has_p4 |= (hm[c0 + i].p == 4);
-    run(pr, "newton_reset", st, [&] { launch_newton_reset(nm, w, st); });
-    run(pr, "newton_bound", st, [&] { launch_newton_bound(A, a_stride, lda, d, nm, eps, w, st); });
-    run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, d, nm, S, eps, w, st); });
-    run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
-    CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
-    CK(cudaEventRecord(ev[0], st));
-    for (int it = 0; it < max_iters; ++it) {
-      // the check of M_it is in flight; queue step it+1 before waiting for it
-      run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, w, st); });
-      if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, w, st); });
-      run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, w, st); });
-      run(pr, "newton_check", st, [&] { launch_newton_check(nm, it + 1, tol, max_iters, w, st); });
-      const int nx = (it + 1) & 1;
+    std::vector<int> done_iters(list.size(), 0);
+    for (int attempt = 0; attempt < kAttempts && !list.empty(); ++attempt) {
+      const int nm = (int)list.size();
+      int has_p4 = 0;
+      for (const auto& m : list) has_p4 |= (m.p == 4);
+      run(pr, "newton_reset", st, [&] { launch_newton_reset(nm, w, st); });
+      run(pr, "newton_bound", st, [&] { launch_newton_bound(A, a_stride, lda, d, nm, eps, attempt, w, st); });
+      run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, d, nm, S, eps, w, st); });
+      run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
+      CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
+      CK(cudaEventRecord(ev[0], st));
+      for (int it = 0; it < max_iters; ++it) {
+        // the check of M_it is in flight; queue step it+1 before waiting for it
+        run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, w, st); });
+        if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, w, st); });
+        run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, w, st); });
+        run(pr, "newton_check", st, [&] { launch_newton_check(nm, it + 1, tol, max_iters, w, st); });
+        const int nx = (it + 1) & 1;
+        CK(cudaGetLastError());
+        CK(cudaMemcpyAsync(&h_count[nx], &w.count[nx], sizeof(int), cudaMemcpyDeviceToHost, st));
+        CK(cudaEventRecord(ev[nx], st));
+        CK(cudaEventSynchronize(ev[it & 1]));
+        if (h_count[it & 1] == 0) break;
+      }
+      CK(cudaMemcpyAsync(hstate.data(), w.state, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
+      CK(cudaMemcpyAsync(hiters.data(), w.iters, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
+      CK(cudaStreamSynchronize(st));
+      std::vector<NewtonMat> again;
+      for (int i = 0; i < nm; ++i)
+        if (hstate[i] == 3) again.push_back(list[i]);
+      const int final_pass = (attempt == kAttempts - 1) || again.empty();
+      run(pr, "newton_finalize", st, [&] {
+        launch_newton_finalize(X, x_stride, ldx, d, nm, S, w, has_root, iters_out, final_pass, st);
+      });
       CK(cudaGetLastError());
-      CK(cudaMemcpyAsync(&h_count[nx], &w.count[nx], sizeof(int), cudaMemcpyDeviceToHost, st));
-      CK(cudaEventRecord(ev[nx], st));
-      CK(cudaEventSynchronize(ev[it & 1]));
-      if (h_count[it & 1] == 0) break;
-    }
-    run(pr, "newton_finalize", st, [&] {
-      launch_newton_finalize(X, x_stride, ldx, d, nm, S, w, has_root, iters_out, st);
-    });
-    CK(cudaGetLastError());
-    CK(cudaMemcpyAsync(hstate.data(), w.state, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
-    CK(cudaMemcpyAsync(hiters.data(), w.iters, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
-    CK(cudaStreamSynchronize(st));
-    for (int i = 0; i < nm; ++i) {
-      if (hstate[i] != 1) ++*n_failed;
-      *max_it = std::max(*max_it, hiters[i]);
-      if (per_matrix) (*per_matrix)[c0 + i] = hstate[i] == 1 ? hiters[i] : -1 - hiters[i];
+      for (int i = 0; i < nm; ++i) {
+        const int slot = list[i].slot;
+        const int k = hiters[i];
+        if (hstate[i] == 1 || hstate[i] == 2 || final_pass) {
+          if (hstate[i] != 1) ++*n_failed;
+          *max_it = std::max(*max_it, k);
+          if (per_slot) (*per_slot)[slot] = hstate[i] == 1 ? k : -1 - k;
+        }
+      }
+      if (final_pass) break;
+      list.swap(again);
+      CK(cudaMemcpyAsync(d_retry, list.data(), list.size() * sizeof(NewtonMat),
+                         cudaMemcpyHostToDevice, st));
+      CK(cudaStreamSynchronize(st));   // list is pageable host memory reused below
+      d = d_retry;
     }
   }
   return SHAMPOO_OK;
@@ -400,7 +430,8 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
              (e = dalloc(ctx, &ctx->flags, (size_t)nparams)) == cudaSuccess &&
              (e = dalloc(ctx, &ctx->has_root, (size_t)ctx->nmat)) == cudaSuccess &&
              (momentum == 0.f || (e = dalloc(ctx, &ctx->mom, (size_t)ctx->total)) == cudaSuccess) &&
-             (e = alloc_newton(ctx, ctx->nw, ctx->newton_chunk, b)) == cudaSuccess;
+             (e = alloc_newton(ctx, ctx->nw, ctx->newton_chunk, b)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->d_retry, (size_t)ctx->newton_chunk)) == cudaSuccess;
   if (!okm) {
     shampoo_destroy(ctx);
     return fail(nullptr, SHAMPOO_ENOMEM, std::string("device allocation failed: ") + cudaGetErrorString(e));
@@ -461,7 +492,8 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
   int nf = 0, mi = 0;
   if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots before update_stats");
   const int64_t slot = (int64_t)ctx->S * ctx->S;
-  shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->stats, slot, ctx->S,
+  shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->d_retry, ctx->stats,
+                                 slot, ctx->S,
                                  ctx->roots, slot, ctx->S, ctx->S, ctx->eps, ctx->tol,
                                  ctx->max_iters, ctx->newton_chunk, ctx->nw, ctx->has_root, nullptr,
                                  ctx->h_count, ctx->ev, ctx->stream, &nf, &mi, &ctx->root_iters);
@@ -611,11 +643,16 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
   std::vector<NewtonMat> hm(batch);
   for (int i = 0; i < batch; ++i) hm[i] = {i, n, p, 0};
   NewtonMat* dm = nullptr;
+  NewtonMat* dr = nullptr;
   NewtonWork w{};
   shampoo_status res = SHAMPOO_OK;
   int nf = 0, mi = 0;
   cudaError_t e = cudaSuccess;
   if ((res = upload(ctx, &dm, hm)) != SHAMPOO_OK) goto done;
+  if ((e = dalloc(ctx, &dr, (size_t)chunk)) != cudaSuccess) {
+    res = fail(ctx, SHAMPOO_ENOMEM, std::string("retry list: ") + cudaGetErrorString(e));
+    goto done;
+  }
   if ((e = alloc_newton(ctx, w, chunk, S)) != cudaSuccess) {
     res = fail(ctx, SHAMPOO_ENOMEM, std::string("work space: ") + cudaGetErrorString(e));
     goto done;
@@ -626,7 +663,7 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
     res = cuda_fail(ctx, e, "set-up");
     goto done;
   }
-  res = run_newton(ctx, nullptr, hm, dm, A, (int64_t)n * n, n, X, (int64_t)n * n, n, S, eps, tol,
+  res = run_newton(ctx, nullptr, hm, dm, dr, A, (int64_t)n * n, n, X, (int64_t)n * n, n, S, eps, tol,
                    max_iters, chunk, w, nullptr, iters, ctx->h_count, ctx->ev, st, &nf, &mi, nullptr);
   if (res == SHAMPOO_OK && nf) res = fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
 done:

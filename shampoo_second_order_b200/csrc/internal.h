@@ -64,19 +64,22 @@ struct NewtonWork {
   double* T2;
   double* T4;
   double* cinv;                 // [nmat] c^{-1}
+  double* ridge;                // [nmat] ridge added to A (eps, raised on a retry)
   unsigned long long* resid;    // [nmat] max|M-I| as ordered bits
   double* prev;                 // [nmat] previous residual
   int* worse;                   // [nmat]
   int* active;                  // [nmat]
   int* iters;                   // [nmat] iterations done
-  int* state;                   // [nmat] 0 running, 1 converged, 2 failed
+  int* state;                   // [nmat] 0 running, 1 converged, 2 failed, 3 diverged
   int* count;                   // [1] matrices still active after a check
 };
 // Set up X0, M0, T0 for `nm` matrices read from `A` (float32, slot-strided
 // `a_stride` elements apart, row stride `lda`, valid side mats[i].size).
 void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s);
+// attempt 0 uses the ridge eps; attempt k > 0 raises it to
+// eps + 8^k 2^-24 c^p (the fp32 resolution of the statistic).
 void launch_newton_bound(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
-                         float eps, NewtonWork w, cudaStream_t s);
+                         float eps, int attempt, NewtonWork w, cudaStream_t s);
 void launch_newton_init(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
                         int S, float eps, NewtonWork w, cudaStream_t s);
 // one Newton step: A (X T and T T), B (T2 T2, p = 4 only), C (T^p M,
@@ -87,8 +90,9 @@ void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, NewtonWo
 void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s);
 // Write the roots back as float32.  keep_old: leave a failed matrix's slot
 // untouched if has_root[slot] is set; else write c^{-1} I.
+// A diverged matrix is skipped unless final_pass (it will be retried).
 void launch_newton_finalize(float* X, int64_t x_stride, int ldx, const NewtonMat* mats, int nm,
-                            int S, NewtonWork w, int* has_root, int32_t* iters_out,
+                            int S, NewtonWork w, int* has_root, int32_t* iters_out, int final_pass,
                             cudaStream_t s);
 
 // ---------------- apply (k_apply.cu) ----------------

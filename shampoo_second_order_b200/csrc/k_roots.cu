@@ -24,7 +24,7 @@ constexpr int kBK = 16;
 constexpr int kAStride = kBK + 4;     // doubles; 4 mod 16 keeps fragment loads conflict-free
 constexpr int kBStride = kTile + 4;
 
-enum : int { kRunning = 0, kConverged = 1, kFailed = 2 };
+enum : int { kRunning = 0, kConverged = 1, kFailed = 2, kDiverged = 3 };
 
 __device__ __forceinline__ unsigned long long dbl_bits(double v) {
   return static_cast<unsigned long long>(__double_as_longlong(v));
@@ -134,10 +134,15 @@ __device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0,
 // ---------------------------------------------------------------------------
 // One CTA per matrix: c^p = min(||A + eps I||_F, ||A + eps I||_inf) over the
 // valid corner.  Both bound the largest eigenvalue of a symmetric matrix.
+// On a retry (attempt k > 0) the ridge is raised to eps + 8^k 2^-24 c^p:
+// rounding of a float32 statistic can leave eigenvalues of A + eps I below
+// zero by about 2^-24 c^p, which the iteration cannot root.
 __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restrict__ A,
                                                            int64_t a_stride, int lda,
                                                            const NewtonMat* __restrict__ mats,
-                                                           float eps, double* __restrict__ cinv,
+                                                           float eps, int attempt,
+                                                           double* __restrict__ cinv,
+                                                           double* __restrict__ ridge,
                                                            double* __restrict__ cpow) {
   __shared__ double red[8];
   const NewtonMat mt = mats[blockIdx.x];
@@ -161,6 +166,13 @@ __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restri
   if (threadIdx.x == 0) {
     double cp = fmin(sqrt(fro), rowmax);
     if (!(cp > 0.0) || !(cp <= DBL_MAX)) cp = (cp > 0.0) ? cp : 1.0;  // NaN/Inf/0 caught later
+    double rd = (double)eps;
+    if (attempt > 0) {
+      const double extra = ldexp(cp, 3 * attempt - 24);
+      rd += extra;
+      cp += extra;   // lambda_max grows by exactly the added ridge
+    }
+    ridge[blockIdx.x] = rd;
     cpow[blockIdx.x] = cp;
     cinv[blockIdx.x] = pow(cp, -1.0 / mt.p);
   }
@@ -171,7 +183,7 @@ __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restri
 __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restrict__ A,
                                                           int64_t a_stride, int lda,
                                                           const NewtonMat* __restrict__ mats,
-                                                          int S, float eps, NewtonWork w,
+                                                          int S, NewtonWork w,
                                                           const double* __restrict__ cpow) {
   __shared__ double red[8];
   const int m = blockIdx.y;
@@ -180,6 +192,7 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
   const int r = blockIdx.x;
   const size_t off = (size_t)m * S * S + (size_t)r * S;
   const double inv_cp = 1.0 / cpow[m];
+  const double rd = w.ridge[m];
   const double ci = w.cinv[m];
   const double pinv = 1.0 / mt.p;
   double dev = 0.0;
@@ -187,7 +200,7 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
     double v;
     if (r < mt.size && c < mt.size) {
       v = (double)a[(size_t)r * lda + c];
-      if (r == c) v += (double)eps;
+      if (r == c) v += rd;
       v *= inv_cp;
     } else {
       v = (r == c) ? 1.0 : 0.0;
@@ -292,9 +305,11 @@ __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, Ne
     const double r = __longlong_as_double(static_cast<long long>(w.resid[m]));
     w.resid[m] = 0ull;
     w.iters[m] = k;
+    // For a PSD A every eigenvalue of M stays in (0, 1], so max|M - I| < 1;
+    // a residual above 1.5 means rounding made A + ridge I indefinite.
     int st = kRunning;
-    if (!(r <= DBL_MAX)) {
-      st = kFailed;
+    if (!(r <= 1.5)) {
+      st = kDiverged;
     } else if (r <= tol) {
       st = kConverged;
     } else if (k >= max_iters) {
@@ -303,7 +318,7 @@ __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, Ne
       const int wo = (r >= w.prev[m]) ? w.worse[m] + 1 : 0;
       w.worse[m] = wo;
       w.prev[m] = r;
-      if (wo >= 5) st = kFailed;
+      if (wo >= 5) st = kDiverged;
     }
     w.state[m] = st;
     alive += (st == kRunning);
@@ -327,10 +342,11 @@ __global__ void newton_reset_kernel(int nm, NewtonWork w) {
 // Failed: keep the old root if there is one, else write c^{-1} I.
 __global__ void __launch_bounds__(256) newton_finalize_kernel(
     float* __restrict__ X, int64_t x_stride, int ldx, const NewtonMat* __restrict__ mats, int S,
-    NewtonWork w, int* __restrict__ has_root, int32_t* __restrict__ iters_out) {
+    NewtonWork w, int* __restrict__ has_root, int32_t* __restrict__ iters_out, int final_pass) {
   const int m = blockIdx.y;
   const NewtonMat mt = mats[m];
   const int st = w.state[m];
+  if (st == kDiverged && !final_pass) return;   // retried with a raised ridge
   const int r = blockIdx.x;
   if (r >= ldx) return;
   const bool ok = (st == kConverged);
@@ -359,13 +375,15 @@ void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s) {
 // c^p goes to the first nm doubles of T2, which no step reads before step A
 // overwrites it.
 void launch_newton_bound(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
-                         float eps, NewtonWork w, cudaStream_t s) {
-  newton_bound_kernel<<<nm, 256, 0, s>>>(A, a_stride, lda, mats, eps, w.cinv, w.T2);
+                         float eps, int attempt, NewtonWork w, cudaStream_t s) {
+  newton_bound_kernel<<<nm, 256, 0, s>>>(A, a_stride, lda, mats, eps, attempt, w.cinv, w.ridge,
+                                         w.T2);
 }
 
 void launch_newton_init(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
                         int S, float eps, NewtonWork w, cudaStream_t s) {
-  newton_init_kernel<<<dim3(S, nm), 256, 0, s>>>(A, a_stride, lda, mats, S, eps, w, w.T2);
+  (void)eps;
+  newton_init_kernel<<<dim3(S, nm), 256, 0, s>>>(A, a_stride, lda, mats, S, w, w.T2);
 }
 
 static int num_tri(int S) {
@@ -390,10 +408,10 @@ void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w,
 }
 
 void launch_newton_finalize(float* X, int64_t x_stride, int ldx, const NewtonMat* mats, int nm,
-                            int S, NewtonWork w, int* has_root, int32_t* iters_out,
+                            int S, NewtonWork w, int* has_root, int32_t* iters_out, int final_pass,
                             cudaStream_t s) {
   newton_finalize_kernel<<<dim3(ldx, nm), 256, 0, s>>>(X, x_stride, ldx, mats, S, w, has_root,
-                                                       iters_out);
+                                                       iters_out, final_pass);
 }
 
 }  // namespace shampoo

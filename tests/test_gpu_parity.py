@@ -4,6 +4,11 @@ Tolerances (relative Frobenius error per object):
   statistics L, R, S              <= 1e-5
   roots, condition number <= 1e6  <= 1e-3
   per block: W_new and the step dW = W_new - W_old   <= 1e-3
+The condition number is that of the oracle's statistic plus eps I.  Beyond
+1e6 the root is not compared: a float32 statistic only resolves eigenvalues
+down to about 2^-24 of its largest, so the root's near-null part is set by
+rounding there; the parameters, which those directions do not reach, are
+still compared.
 Both sides take the same seeded inputs from the workloads module; the oracle
 never sees a value the CUDA path produced except where a test compares.
 """
@@ -75,6 +80,9 @@ def run_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, interval, seed
             for k in range(opt.num_matrices()):
                 S, _ = opt.read_matrix(0, k)
                 worst["stats"] = max(worst["stats"], rel(S, mats[k][0]))
+                ev = np.linalg.eigvalsh(mats[k][0]) + eps
+                if ev.max() / max(ev.min(), 1e-300) > 1e6:
+                    continue
                 X, _ = opt.read_matrix(1, k)
                 worst["roots"] = max(worst["roots"], rel(X, ro[k]))
         for i, s in enumerate(shapes):
@@ -218,9 +226,9 @@ def test_apply_before_roots_is_state_error():
 
 def test_iteration_cap_reports_not_converged_and_falls_back():
     from shampoo_second_order_b200 import Shampoo
-    opt = Shampoo([(64, 32)], 64, 1.0, 1e-6)
+    opt = Shampoo([(64, 64)], 64, 1.0, 1e-6)    # square gradient: L and R full rank
     opt.set_root_options(1e-6, 2)
-    g = [torch.randn(64, 32, device="cuda")]
+    g = [torch.randn(64, 64, device="cuda")]
     opt.update_stats(g)
     assert opt.compute_roots() is False
     nf, it = opt.root_status()
