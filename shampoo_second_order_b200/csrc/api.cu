@@ -1,6 +1,8 @@
 // C-ABI of the library (include/shampoo.h): the host-side planner that builds
 // the block table, owns the device state and sequences the kernels of one
 // optimizer step on the caller's stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -109,6 +111,7 @@ struct shampoo_ctx {
   std::vector<BlockDesc> blocks;
   std::vector<SegDesc> segs;
   std::vector<ChunkDesc> chunks;
+  std::vector<ChunkDesc> chunks1d;   // chunks of the 1-D parameters only
   std::vector<NewtonMat> mats;
   int64_t total = 0;
   int nmat = 0;
@@ -118,6 +121,7 @@ struct shampoo_ctx {
   BlockDesc* d_blocks = nullptr;
   SegDesc* d_segs = nullptr;
   ChunkDesc* d_chunks = nullptr;
+  ChunkDesc* d_chunks1d = nullptr;
   NewtonMat* d_mats = nullptr;
   const void** d_gptr = nullptr;
   float** d_wptr = nullptr;
@@ -126,8 +130,16 @@ struct shampoo_ctx {
   float* a = nullptr;
   float* mom = nullptr;
   float* P = nullptr;
-  float* Y = nullptr;
-  double* norms = nullptr;
+  uint16_t* gblk = nullptr;     // gathered gradient planes [planes_g*nblk][S][S] (h, m, l)
+  uint16_t* rplanes = nullptr;  // root planes [2*nmat][S][S]
+  uint16_t* yplanes = nullptr;  // Y planes [2*nblk][S][S]
+  TcMaps maps{};
+  int planes_g = 1;
+  int* d_err = nullptr;
+  std::vector<const void*> gathered_from;   // gradient pointers of the last gather
+  std::vector<const void*> stats_from;      // gradient pointers of the last update_stats
+  double* d2 = nullptr;   // [nparams] ||D||^2 of the graft target
+  double* p2 = nullptr;   // [nparams] ||P||^2
   int* flags = nullptr;
   int* has_root = nullptr;
   NewtonWork nw{};
@@ -214,7 +226,7 @@ constexpr int kAttempts = 4;
 
 shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<NewtonMat>& hm,
                           const NewtonMat* dm, NewtonMat* d_retry, const float* A,
-                          int64_t a_stride, int lda, float* X, int64_t x_stride, int ldx, int S,
+                          int64_t a_stride, int lda, int upper, float* X, int64_t x_stride, int ldx, int S,
                           float eps, double tol, int max_iters, int chunk, NewtonWork& w,
                           int* has_root, int32_t* iters_out, int* h_count, cudaEvent_t* ev,
                           cudaStream_t st, int* n_failed, int* max_it,
@@ -235,8 +247,10 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
       int has_p4 = 0;
       for (const auto& m : list) has_p4 |= (m.p == 4);
       run(pr, "newton_reset", st, [&] { launch_newton_reset(nm, w, st); });
-      run(pr, "newton_bound", st, [&] { launch_newton_bound(A, a_stride, lda, d, nm, eps, attempt, w, st); });
-      run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, d, nm, S, eps, w, st); });
+      run(pr, "newton_bound", st, [&] {
+        launch_newton_bound(A, a_stride, lda, upper, d, nm, eps, attempt, w, st);
+      });
+      run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, upper, d, nm, S, w, st); });
       run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
       CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
       CK(cudaEventRecord(ev[0], st));
@@ -300,6 +314,59 @@ shampoo_status set_pointers(shampoo_ctx* ctx, const void* const* grads, float* c
   return SHAMPOO_OK;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor [depth][S][S] with a box of box_x (inner) x box_y rows.
+bool encode_planes(CUtensorMap* m, void* base, int S, int64_t depth, int box_x, int box_y) {
+  auto fn = encode_fn();
+  if (!fn || depth < 1) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)S, (cuuint64_t)S, (cuuint64_t)depth};
+  cuuint64_t strides[2] = {(cuuint64_t)S * 2, (cuuint64_t)S * S * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A kernel that gave up on a wait leaves a code in the error word.
+shampoo_status check_kernel_error(shampoo_ctx* ctx) {
+  int e = 0;
+  CK(cudaMemcpyAsync(&e, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost, ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  if (e) return fail(ctx, SHAMPOO_ECUDA, "a tensor-core kernel timed out waiting on its pipeline");
+  return SHAMPOO_OK;
+}
+
+// Gather the 2-D gradients into the blocked bf16 planes unless the planes
+// already hold these very gradient pointers from this step's update_stats.
+shampoo_status gather(shampoo_ctx* ctx, const void* const* grads, bool force) {
+  const int nblk = (int)ctx->blocks.size();
+  if (!nblk) return SHAMPOO_OK;
+  bool same = !force && ctx->gathered_from.size() == (size_t)ctx->nparams;
+  for (int i = 0; same && i < ctx->nparams; ++i) same = ctx->gathered_from[i] == grads[i];
+  if (same) return SHAMPOO_OK;
+  cudaError_t e = cudaSuccess;
+  run(&ctx->prof, "gather", ctx->stream, [&] {
+    e = launch_gather(ctx->d_blocks, nblk, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->S, ctx->gblk,
+                      ctx->stream);
+  });
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "gather");
+  ctx->gathered_from.assign(grads, grads + ctx->nparams);
+  return SHAMPOO_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -348,6 +415,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   ctx->mu = momentum;
   ctx->graft = graft;
   ctx->bf16 = grad_dtype == SHAMPOO_BF16;
+  ctx->planes_g = ctx->bf16 ? 1 : 3;
   const int b = block_size;
 
   for (int i = 0; i < nparams; ++i) {
@@ -383,6 +451,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
       ch.start = s0;
       ch.len = (int)std::min<int64_t>(kChunk, pd.numel - s0);
       ctx->chunks.push_back(ch);
+      if (nd == 1) ctx->chunks1d.push_back(ch);
     }
   }
   for (int i = 0; i < nparams; ++i) {
@@ -409,12 +478,14 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
       (st = upload(ctx, &ctx->d_blocks, ctx->blocks)) != SHAMPOO_OK ||
       (st = upload(ctx, &ctx->d_segs, ctx->segs)) != SHAMPOO_OK ||
       (st = upload(ctx, &ctx->d_chunks, ctx->chunks)) != SHAMPOO_OK ||
+      (st = upload(ctx, &ctx->d_chunks1d, ctx->chunks1d)) != SHAMPOO_OK ||
       (st = upload(ctx, &ctx->d_mats, ctx->mats)) != SHAMPOO_OK) {
     g_create_err = ctx->err;
     shampoo_destroy(ctx);
     return st;
   }
   const size_t slot = (size_t)b * b;
+  const int64_t nblk64 = (int64_t)ctx->blocks.size();
   // Newton work space: at most ~4 GiB of float64 in flight.
   const size_t per = 7 * slot * sizeof(double);
   ctx->newton_chunk = (int)std::max<size_t>(1, std::min<size_t>(ctx->nmat, (size_t(4) << 30) / per));
@@ -425,13 +496,17 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
              (e = dalloc(ctx, &ctx->roots, ctx->nmat * slot)) == cudaSuccess &&
              (e = dalloc(ctx, &ctx->a, (size_t)ctx->total)) == cudaSuccess &&
              (e = dalloc(ctx, &ctx->P, (size_t)ctx->total)) == cudaSuccess &&
-             (e = dalloc(ctx, &ctx->Y, ctx->blocks.size() * slot)) == cudaSuccess &&
-             (e = dalloc(ctx, &ctx->norms, 2 * (size_t)nparams)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->d2, (size_t)nparams)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->p2, (size_t)nparams)) == cudaSuccess &&
              (e = dalloc(ctx, &ctx->flags, (size_t)nparams)) == cudaSuccess &&
              (e = dalloc(ctx, &ctx->has_root, (size_t)ctx->nmat)) == cudaSuccess &&
              (momentum == 0.f || (e = dalloc(ctx, &ctx->mom, (size_t)ctx->total)) == cudaSuccess) &&
              (e = alloc_newton(ctx, ctx->nw, ctx->newton_chunk, b)) == cudaSuccess &&
-             (e = dalloc(ctx, &ctx->d_retry, (size_t)ctx->newton_chunk)) == cudaSuccess;
+             (e = dalloc(ctx, &ctx->d_retry, (size_t)ctx->newton_chunk)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->d_err, 1)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->gblk, (size_t)ctx->planes_g * ctx->blocks.size() * slot)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->rplanes, 2 * (size_t)ctx->nmat * slot)) == cudaSuccess &&
+             (e = dalloc(ctx, &ctx->yplanes, 2 * ctx->blocks.size() * slot)) == cudaSuccess;
   if (!okm) {
     shampoo_destroy(ctx);
     return fail(nullptr, SHAMPOO_ENOMEM, std::string("device allocation failed: ") + cudaGetErrorString(e));
@@ -445,11 +520,24 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->P, 0, ctx->total * sizeof(float), ctx->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->flags, 0, nparams * sizeof(int), ctx->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->has_root, 0, ctx->nmat * sizeof(int), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->d_err, 0, sizeof(int), ctx->stream);
+  if (e == cudaSuccess && nblk64)
+    e = cudaMemsetAsync(ctx->gblk, 0, ctx->planes_g * nblk64 * slot * 2, ctx->stream);
+  if (e == cudaSuccess && nblk64) e = cudaMemsetAsync(ctx->yplanes, 0, 2 * nblk64 * slot * 2, ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->rplanes, 0, 2 * (size_t)ctx->nmat * slot * 2, ctx->stream);
   if (e == cudaSuccess && ctx->mom) e = cudaMemsetAsync(ctx->mom, 0, ctx->total * sizeof(float), ctx->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
   if (e != cudaSuccess) {
     shampoo_destroy(ctx);
     return fail(nullptr, SHAMPOO_ECUDA, std::string("state set-up failed: ") + cudaGetErrorString(e));
+  }
+  if (nblk64 &&
+      !(encode_planes(&ctx->maps.gk, ctx->gblk, b, ctx->planes_g * nblk64, 64, 128) &&
+        encode_planes(&ctx->maps.gmn, ctx->gblk, b, ctx->planes_g * nblk64, 64, 64) &&
+        encode_planes(&ctx->maps.rk, ctx->rplanes, b, 2 * (int64_t)ctx->nmat, 64, 128) &&
+        encode_planes(&ctx->maps.ymn, ctx->yplanes, b, 2 * nblk64, 64, 64))) {
+    shampoo_destroy(ctx);
+    return fail(nullptr, SHAMPOO_ECUDA, "cuTensorMapEncodeTiled failed");
   }
   *out = ctx;
   return SHAMPOO_OK;
@@ -464,19 +552,32 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
   const int nblk = (int)ctx->blocks.size(), nseg = (int)ctx->segs.size();
   Profiler* pr = &ctx->prof;
   CK(cudaMemsetAsync(ctx->flags, 0, ctx->nparams * sizeof(int), s));
-  run(pr, "check_finite", s, [&] {
-    launch_check_finite(ctx->d_chunks, nch, ctx->d_gptr, ctx->bf16, ctx->flags, s);
-  });
-  if (ctx->graft)
+  // the non-finite check: 1-D gradients here, 2-D ones inside the gather
+  const int nch1 = (int)ctx->chunks1d.size();
+  if (nch1)
+    run(pr, "check_finite", s, [&] {
+      launch_check_finite(ctx->d_chunks1d, nch1, ctx->d_gptr, ctx->bf16, ctx->flags, s);
+    });
+  if (nblk) {
+    shampoo_status gs = gather(ctx, grads, true);
+    if (gs != SHAMPOO_OK) return gs;
+  }
+  if (ctx->graft) {
+    CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), s));
     run(pr, "diag_update", s, [&] {
       launch_diag_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags,
-                         ctx->beta2, ctx->a, s);
+                         ctx->beta2, ctx->eps, ctx->a, ctx->d2, s);
     });
-  if (nblk)
-    run(pr, "stats_blocks", s, [&] {
-      launch_stats_blocks(ctx->d_blocks, nblk, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->beta2,
-                          ctx->stats, ctx->S, s);
+  }
+  ctx->stats_from.assign(grads, grads + ctx->nparams);
+  if (nblk) {
+    cudaError_t e = cudaSuccess;
+    run(pr, "stats_tc", s, [&] {
+      e = launch_stats_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S,
+                          ctx->planes_g, ctx->beta2, ctx->stats, ctx->d_err, s);
     });
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "stats_tc");
+  }
   if (nseg)
     run(pr, "stats_segments", s, [&] {
       launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
@@ -493,11 +594,16 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
   if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots before update_stats");
   const int64_t slot = (int64_t)ctx->S * ctx->S;
   shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->d_retry, ctx->stats,
-                                 slot, ctx->S,
+                                 slot, ctx->S, 1,
                                  ctx->roots, slot, ctx->S, ctx->S, ctx->eps, ctx->tol,
                                  ctx->max_iters, ctx->newton_chunk, ctx->nw, ctx->has_root, nullptr,
                                  ctx->h_count, ctx->ev, ctx->stream, &nf, &mi, &ctx->root_iters);
   if (st != SHAMPOO_OK) return st;
+  cudaError_t e = cudaSuccess;
+  run(&ctx->prof, "split_roots", ctx->stream, [&] {
+    e = launch_split(ctx->roots, (int64_t)ctx->nmat * slot, ctx->rplanes, ctx->stream);
+  });
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "split_roots");
   ctx->roots_done = true;
   ctx->last_not_converged = nf;
   ctx->last_max_iters = mi;
@@ -517,30 +623,39 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
   const int nblk = (int)ctx->blocks.size();
   const int nseg = (int)ctx->segs.size();
   Profiler* pr = &ctx->prof;
-  CK(cudaMemsetAsync(ctx->norms, 0, 2 * ctx->nparams * sizeof(double), s));
-  if (ctx->graft)
+  CK(cudaMemsetAsync(ctx->p2, 0, ctx->nparams * sizeof(double), s));
+  bool same = ctx->stats_from.size() == (size_t)ctx->nparams;
+  for (int i = 0; same && i < ctx->nparams; ++i) same = ctx->stats_from[i] == grads[i];
+  if (ctx->graft && !same) {   // ||D||^2 of these gradients against the current a
+    CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), s));
     run(pr, "dnorm", s, [&] {
       launch_dnorm(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->a,
-                   ctx->eps, ctx->norms, s);
+                   ctx->eps, ctx->d2, s);
     });
+  }
   if (nblk) {
-    run(pr, "precond_y", s, [&] {
-      launch_precond_y(ctx->d_blocks, nblk, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->roots, ctx->S,
-                       ctx->Y, s);
+    shampoo_status gs = gather(ctx, grads, false);
+    if (gs != SHAMPOO_OK) return gs;
+    cudaError_t e = cudaSuccess;
+    run(pr, "apply_y_tc", s, [&] {
+      e = launch_apply_y_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S,
+                            ctx->planes_g, ctx->yplanes, ctx->d_err, s);
     });
-    run(pr, "precond_p", s, [&] {
-      launch_precond_p(ctx->d_blocks, nblk, ctx->d_params, ctx->flags, ctx->roots, ctx->S, ctx->Y,
-                       ctx->P, ctx->norms, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "apply_y_tc");
+    run(pr, "apply_p_tc", s, [&] {
+      e = launch_apply_p_tc(ctx->maps, ctx->d_blocks, ctx->d_params, ctx->flags, nblk, ctx->nmat,
+                            ctx->S, ctx->P, ctx->p2, ctx->d_err, s);
     });
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "apply_p_tc");
   }
   if (nseg)
     run(pr, "precond_seg", s, [&] {
       launch_precondition_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_params, ctx->d_gptr,
-                                   ctx->bf16, ctx->flags, ctx->roots, ctx->S, ctx->P, ctx->norms, s);
+                                   ctx->bf16, ctx->flags, ctx->roots, ctx->S, ctx->P, ctx->p2, s);
     });
   run(pr, "update", s, [&] {
-    launch_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_wptr, ctx->flags, ctx->P, ctx->norms,
-                  ctx->graft, ctx->mu, lr, ctx->mom, s);
+    launch_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_wptr, ctx->flags, ctx->P, ctx->d2,
+                  ctx->p2, ctx->graft, ctx->mu, lr, ctx->mom, s);
   });
   CK(cudaGetLastError());
   return SHAMPOO_OK;
@@ -548,7 +663,8 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
 
 shampoo_status shampoo_root_status(shampoo_ctx* ctx, int* n_not_converged, int* max_iters) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
-  CK(cudaStreamSynchronize(ctx->stream));
+  shampoo_status ks = check_kernel_error(ctx);
+  if (ks != SHAMPOO_OK) return ks;
   if (n_not_converged) *n_not_converged = ctx->last_not_converged;
   if (max_iters) *max_iters = ctx->last_max_iters;
   return SHAMPOO_OK;
@@ -560,7 +676,8 @@ shampoo_status shampoo_nonfinite_status(shampoo_ctx* ctx, int* n_params_skipped)
   std::vector<int> f(ctx->nparams);
   CK(cudaMemcpyAsync(f.data(), ctx->flags, ctx->nparams * sizeof(int), cudaMemcpyDeviceToHost,
                      ctx->stream));
-  CK(cudaStreamSynchronize(ctx->stream));
+  shampoo_status ks = check_kernel_error(ctx);
+  if (ks != SHAMPOO_OK) return ks;
   int n = 0;
   for (int v : f) n += v != 0;
   *n_params_skipped = n;
@@ -591,8 +708,17 @@ shampoo_status shampoo_read_matrix(shampoo_ctx* ctx, int which, int index, float
     return fail(ctx, SHAMPOO_EINVAL, "bad which / index / dst");
   const size_t slot = (size_t)ctx->S * ctx->S;
   const float* src = (which == 0 ? ctx->stats : ctx->roots) + slot * index;
-  CK(cudaMemcpyAsync(dst, src, slot * sizeof(float), cudaMemcpyDefault, ctx->stream));
+  std::vector<float> h(slot);
+  CK(cudaMemcpyAsync(h.data(), src, slot * sizeof(float), cudaMemcpyDeviceToHost, ctx->stream));
   CK(cudaStreamSynchronize(ctx->stream));
+  // block statistics keep only their upper 128 x 128 tiles: mirror the rest
+  if (which == 0 && index < 2 * (int)ctx->blocks.size()) {
+    const int S = ctx->S;
+    for (int r = 0; r < S; ++r)
+      for (int c = 0; c < S; ++c)
+        if ((r >> 7) > (c >> 7)) h[(size_t)r * S + c] = h[(size_t)c * S + r];
+  }
+  CK(cudaMemcpy(dst, h.data(), slot * sizeof(float), cudaMemcpyDefault));
   return SHAMPOO_OK;
 }
 
@@ -663,7 +789,7 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
     res = cuda_fail(ctx, e, "set-up");
     goto done;
   }
-  res = run_newton(ctx, nullptr, hm, dm, dr, A, (int64_t)n * n, n, X, (int64_t)n * n, n, S, eps, tol,
+  res = run_newton(ctx, nullptr, hm, dm, dr, A, (int64_t)n * n, n, 0, X, (int64_t)n * n, n, S, eps, tol,
                    max_iters, chunk, w, nullptr, iters, ctx->h_count, ctx->ev, st, &nf, &mi, nullptr);
   if (res == SHAMPOO_OK && nf) res = fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
 done:

@@ -58,53 +58,4 @@ __device__ __forceinline__ double block_max(double v, double* red) {
   return s;
 }
 
-// A strided read-only view of a matrix: element (i, k) is p[i*si + k*sk]
-// when i < mi and k < mk, and 0 outside (the zero padding of ragged blocks).
-struct View {
-  const void* p;
-  int64_t si, sk;
-  int mi, mk;
-  int bf16;
-};
-
-__device__ __forceinline__ float view_at(const View& v, int i, int k) {
-  if (i < v.mi && k < v.mk) return grad_at(v.p, i * v.si + k * v.sk, v.bf16);
-  return 0.0f;
-}
-
-// One 64 x 64 fp32 output tile, C(i, j) = sum_k A(i, k) * Bt(j, k), on 256
-// threads; thread (ty, tx) = (t / 16, t % 16) owns rows ty*4.., cols tx*4..
-// The loads follow whichever stride of the view is 1, so each warp reads
-// contiguous memory.  Exact fp32 FMA products and sums.
-__device__ __forceinline__ void tile_gemm_f32(const View& A, const View& B, int i0, int j0,
-                                              int K, float acc[4][4], float (*As)[68],
-                                              float (*Bs)[68]) {
-  const int t = threadIdx.x;
-  const int ty = t >> 4, tx = t & 15;
-  for (int k0 = 0; k0 < K; k0 += 16) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int e = t + r * 256;
-      int i, k;
-      if (A.sk == 1) { k = e & 15; i = e >> 4; } else { i = e & 63; k = e >> 6; }
-      As[k][i] = view_at(A, i0 + i, k0 + k);
-      if (B.sk == 1) { k = e & 15; i = e >> 4; } else { i = e & 63; k = e >> 6; }
-      Bs[k][i] = view_at(B, j0 + i, k0 + k);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
-    }
-    __syncthreads();
-  }
-}
-
 }  // namespace shampoo

@@ -1,5 +1,6 @@
 // Internal declarations shared by the host planner and the kernels.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -44,14 +45,36 @@ struct NewtonMat {
   int pad;
 };
 
+// TMA descriptors of the library's bf16 operand planes (128-byte swizzle):
+//  gk   gathered gradient blocks [planes*nblk][S][S], box 64 x 128 (K-major)
+//  gmn  the same tensor, box 64 x 64 (MN-major loads of G^T)
+//  rk   root planes [2*nmat][S][S] (hi then lo), box 64 x 128
+//  ymn  Y = G R^{-1/p} planes [2*nblk][S][S], box 64 x 64 (MN-major)
+struct TcMaps {
+  CUtensorMap gk, gmn, rk, ymn;
+};
+
+// ---------------- tensor-core kernels (k_tc.cu) ----------------
+// also flags (atomically) a parameter whose gradient holds NaN or Inf
+cudaError_t launch_gather(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
+                          int* flags, int S, uint16_t* out, cudaStream_t s);
+cudaError_t launch_split(const float* x, int64_t n, uint16_t* out, cudaStream_t s);
+cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
+                            int nmat, int S, int planes_g, float beta2, float* stats, int* err,
+                            cudaStream_t s);
+cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
+                              int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s);
+cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const ParamDesc* params,
+                              const int* flags, int nblk, int nmat, int S, float* P, double* p2,
+                              int* err, cudaStream_t s);
+
 // ---------------- stats (k_stats.cu) ----------------
 void launch_check_finite(const ChunkDesc* chunks, int nchunks, const void* const* gptr,
                          int bf16, int* flags, cudaStream_t s);
+// a <- beta2 a + g*g, and d2[param] += sum (g / sqrt(a + eps))^2
 void launch_diag_update(const ChunkDesc* chunks, int nchunks, const ParamDesc* params,
-                        const void* const* gptr, int bf16, const int* flags, float beta2,
-                        float* a, cudaStream_t s);
-void launch_stats_blocks(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
-                         const int* flags, float beta2, float* stats, int S, cudaStream_t s);
+                        const void* const* gptr, int bf16, const int* flags, float beta2, float eps,
+                        float* a, double* d2, cudaStream_t s);
 void launch_stats_segments(const SegDesc* segs, int nseg, int mat0, const void* const* gptr,
                            int bf16, const int* flags, float beta2, float* stats, int S,
                            cudaStream_t s);
@@ -78,10 +101,12 @@ struct NewtonWork {
 void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s);
 // attempt 0 uses the ridge eps; attempt k > 0 raises it to
 // eps + 8^k 2^-24 c^p (the fp32 resolution of the statistic).
-void launch_newton_bound(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
-                         float eps, int attempt, NewtonWork w, cudaStream_t s);
-void launch_newton_init(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
-                        int S, float eps, NewtonWork w, cudaStream_t s);
+// upper: A holds only its upper-triangular 128 x 128 tiles; element (r, c)
+// of a lower tile is read from (c, r).
+void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                         int nm, float eps, int attempt, NewtonWork w, cudaStream_t s);
+void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                        int nm, int S, NewtonWork w, cudaStream_t s);
 // one Newton step: A (X T and T T), B (T2 T2, p = 4 only), C (T^p M,
 // residual, next T); check k: convergence test of M_k
 void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);
@@ -98,18 +123,13 @@ void launch_newton_finalize(float* X, int64_t x_stride, int ldx, const NewtonMat
 // ---------------- apply (k_apply.cu) ----------------
 void launch_dnorm(const ChunkDesc* chunks, int nchunks, const ParamDesc* params,
                   const void* const* gptr, int bf16, const int* flags, const float* a, float eps,
-                  double* norms, cudaStream_t s);
-void launch_precond_y(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
-                      const int* flags, const float* roots, int S, float* Y, cudaStream_t s);
-void launch_precond_p(const BlockDesc* blocks, int nblk, const ParamDesc* params, const int* flags,
-                      const float* roots, int S, const float* Y, float* P, double* norms,
-                      cudaStream_t s);
+                  double* d2, cudaStream_t s);
 void launch_precondition_segments(const SegDesc* segs, int nseg, int mat0, const ParamDesc* params,
                                   const void* const* gptr, int bf16, const int* flags,
-                                  const float* roots, int S, float* P, double* norms,
+                                  const float* roots, int S, float* P, double* p2,
                                   cudaStream_t s);
 void launch_update(const ChunkDesc* chunks, int nchunks, const ParamDesc* params, float* const* wptr,
-                   const int* flags, const float* P, const double* norms, int graft, float mu,
-                   float lr, float* mom, cudaStream_t s);
+                   const int* flags, const float* P, const double* d2, const double* p2, int graft,
+                   float mu, float lr, float* mom, cudaStream_t s);
 
 }  // namespace shampoo

@@ -137,8 +137,13 @@ __device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0,
 // On a retry (attempt k > 0) the ridge is raised to eps + 8^k 2^-24 c^p:
 // rounding of a float32 statistic can leave eigenvalues of A + eps I below
 // zero by about 2^-24 c^p, which the iteration cannot root.
+__device__ __forceinline__ float sym_at(const float* a, int lda, int upper, int r, int c) {
+  if (upper && (r >> 7) > (c >> 7)) return a[(size_t)c * lda + r];
+  return a[(size_t)r * lda + c];
+}
+
 __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restrict__ A,
-                                                           int64_t a_stride, int lda,
+                                                           int64_t a_stride, int lda, int upper,
                                                            const NewtonMat* __restrict__ mats,
                                                            float eps, int attempt,
                                                            double* __restrict__ cinv,
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restri
   for (int r = warp; r < n; r += 8) {
     double rs = 0.0;
     for (int c = lane; c < n; c += 32) {
-      double v = (double)a[(size_t)r * lda + c];
+      double v = (double)sym_at(a, lda, upper, r, c);
       if (r == c) v += (double)eps;
       rs += fabs(v);
       fro += v * v;
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restri
 // grid: x = row of the S x S slot, y = matrix.  Writes X0, M0, T0 into the
 // parity-0 buffers and folds max|M0 - I| into the residual.
 __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restrict__ A,
-                                                          int64_t a_stride, int lda,
+                                                          int64_t a_stride, int lda, int upper,
                                                           const NewtonMat* __restrict__ mats,
                                                           int S, NewtonWork w,
                                                           const double* __restrict__ cpow) {
@@ -199,7 +204,7 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
   for (int c = threadIdx.x; c < S; c += blockDim.x) {
     double v;
     if (r < mt.size && c < mt.size) {
-      v = (double)a[(size_t)r * lda + c];
+      v = (double)sym_at(a, lda, upper, r, c);
       if (r == c) v += rd;
       v *= inv_cp;
     } else {
@@ -374,16 +379,15 @@ void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s) {
 
 // c^p goes to the first nm doubles of T2, which no step reads before step A
 // overwrites it.
-void launch_newton_bound(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
-                         float eps, int attempt, NewtonWork w, cudaStream_t s) {
-  newton_bound_kernel<<<nm, 256, 0, s>>>(A, a_stride, lda, mats, eps, attempt, w.cinv, w.ridge,
-                                         w.T2);
+void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                         int nm, float eps, int attempt, NewtonWork w, cudaStream_t s) {
+  newton_bound_kernel<<<nm, 256, 0, s>>>(A, a_stride, lda, upper, mats, eps, attempt, w.cinv,
+                                         w.ridge, w.T2);
 }
 
-void launch_newton_init(const float* A, int64_t a_stride, int lda, const NewtonMat* mats, int nm,
-                        int S, float eps, NewtonWork w, cudaStream_t s) {
-  (void)eps;
-  newton_init_kernel<<<dim3(S, nm), 256, 0, s>>>(A, a_stride, lda, mats, S, w, w.T2);
+void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                        int nm, int S, NewtonWork w, cudaStream_t s) {
+  newton_init_kernel<<<dim3(S, nm), 256, 0, s>>>(A, a_stride, lda, upper, mats, S, w, w.T2);
 }
 
 static int num_tri(int S) {

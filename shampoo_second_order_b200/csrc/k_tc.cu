@@ -1,0 +1,429 @@
+// Tensor-core (tcgen05) kernels of the step:
+//   gather   K1: partition each 2-D gradient into zero-padded S x S blocks as
+//                bf16 planes (fp32 gradients: hi = bf16(g), lo = bf16(g - hi))
+//   stats    K2: L <- beta2 L + G G^T, R <- beta2 R + G^T G (transcript
+//                segment 10, first piece), upper-triangular 128 x 128 tiles
+//   apply    K4: Y = G R^{-1/p}, then P = L^{-1/p} Y (segment 10, third piece)
+//   split        roots (fp32) -> bf16 hi/lo planes for the apply GEMMs
+//
+// Every product runs as bf16 x bf16 -> fp32 on tcgen05 with the accumulator
+// in TMEM; fp32 operands enter as sums of bf16 terms.  bf16 gradients are
+// exact in one term.  fp32 gradients are split into three terms x = h + m + l
+// (24 significant bits, exact for normal floats) and the statistics keep the
+// six products h h, h m, m h, h l, m m, l h, dropping only terms below
+// 2^-24 |x||y|: a statistic of an ill-conditioned block amplifies its own
+// error by up to its condition number in the root, so L and R need fp32
+// accuracy.  The apply products keep hi*hi + hi*lo + lo*hi of two-term
+// splits (relative error near 2^-16), well inside the step tolerance.
+//
+// One CTA computes one 128 x 128 output tile with 128 threads: lane 0 of
+// warp 0 issues TMA loads into a ring of shared-memory stages, lane 0 of warp
+// 1 issues the MMAs and releases stages through tcgen05.commit, and all four
+// warps then read the accumulator out of TMEM (warp w owns rows 32w..32w+31).
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace shampoo {
+
+namespace {
+
+constexpr int kTM = 128;          // output tile side (M = N = 128)
+constexpr int kBKe = 64;          // K elements per stage (one 128-byte row)
+constexpr int kBoxBytes = kTM * kBKe * 2;   // 16 KB: one operand plane per stage
+
+enum : int { kStats = 0, kApplyY = 1, kApplyP = 2 };
+
+struct TcArgs {
+  const BlockDesc* blocks;
+  const ParamDesc* params;
+  const int* flags;
+  int nblk, nmat, S;
+  int planes_g;      // 1: bf16 gradients, 3: fp32 gradients (h, m, l)
+  float beta2;
+  float* stats;      // fp32 [nmat][S][S], upper 128-tiles kept
+  uint16_t* y;       // bf16 planes [2][nblk][S][S], row-major Y
+  float* P;          // parameter-shaped preconditioned gradient
+  double* p2;        // [nparams] sum of P^2
+  int* err;
+};
+
+__device__ __forceinline__ void tri_tile128(int idx, int T, int& ti, int& tj) {
+  ti = 0;
+  while (idx >= T - ti) {
+    idx -= T - ti;
+    ++ti;
+  }
+  tj = ti + idx;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap map_gk,
+                                                         const __grid_constant__ CUtensorMap map_gmn,
+                                                         const __grid_constant__ CUtensorMap map_rk,
+                                                         const __grid_constant__ CUtensorMap map_ymn,
+                                                         TcArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int blk = blockIdx.y;
+  const BlockDesc bd = args.blocks[blk];
+  if (args.flags[bd.param]) return;
+  const int S = args.S;
+  const int T = (S + kTM - 1) / kTM;
+
+  // ---- what this CTA computes ----
+  int ti, tj, K, a_mn = 0, b_mn = 0, isR = 0;
+  if (MODE == kStats) {
+    isR = blockIdx.z;
+    tri_tile128(blockIdx.x, T, ti, tj);
+    const int side = isR ? bd.n : bd.m;
+    if (ti * kTM >= side || tj * kTM >= side) return;
+    K = isR ? bd.m : bd.n;
+    a_mn = b_mn = isR;
+  } else {
+    ti = blockIdx.x / T;
+    tj = blockIdx.x % T;
+    if (ti * kTM >= bd.m || tj * kTM >= bd.n) return;
+    K = (MODE == kApplyY) ? bd.n : bd.m;
+    b_mn = (MODE == kApplyP);
+  }
+  const int i0 = ti * kTM, j0 = tj * kTM;
+  const int nk = (K + kBKe - 1) / kBKe;
+  // operand planes loaded and the (A plane, B plane) products kept, packed
+  // two bits per product
+  const bool g1 = args.planes_g == 1;
+  const int nA = (MODE == kApplyP) ? 2 : (MODE == kApplyY ? (g1 ? 1 : 2) : args.planes_g);
+  const int nB = (MODE == kStats) ? args.planes_g : 2;
+  int npass;
+  uint32_t pas, pbs;
+  if (MODE == kStats && g1) {
+    npass = 1; pas = 0; pbs = 0;                          // g g
+  } else if (MODE == kStats) {
+    npass = 6;                                            // hh hm mh hl mm lh
+    pas = (0u) | (0u << 2) | (1u << 4) | (0u << 6) | (1u << 8) | (2u << 10);
+    pbs = (0u) | (1u << 2) | (0u << 4) | (2u << 6) | (1u << 8) | (0u << 10);
+  } else if (MODE == kApplyY && g1) {
+    npass = 2; pas = 0; pbs = (1u << 2);                  // g R_h, g R_l
+  } else {
+    npass = 3; pas = (1u << 4); pbs = (1u << 2);          // h h, h l, l h
+  }
+  const int stage_bytes = (nA + nB) * kBoxBytes;
+  const int ST = stage_bytes <= 3 * kBoxBytes ? 3 : 2;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * stage_bytes);
+  uint64_t* empty = full + ST;
+  uint64_t* accum = empty + ST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (tid == 0) {
+    for (int s = 0; s < ST; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(accum, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tmem_slot, 128);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    const CUtensorMap* mA = (MODE == kApplyP) ? &map_rk : (isR ? &map_gmn : &map_gk);
+    const CUtensorMap* mB = (MODE == kStats) ? (isR ? &map_gmn : &map_gk)
+                                             : (MODE == kApplyY ? &map_rk : &map_ymn);
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % ST;
+      if (kt >= ST && !tc::mbar_wait(&empty[s], ((kt / ST) - 1) & 1)) {
+        *abort_flag = 1;
+        atomicExch(args.err, tc::kErrTimeout);
+        break;
+      }
+      uint8_t* st = smem + s * stage_bytes;
+      tc::mbar_expect_tx(&full[s], stage_bytes);
+      const int k0 = kt * kBKe;
+      for (int pa = 0; pa < nA; ++pa) {
+        uint8_t* dst = st + pa * kBoxBytes;
+        if (MODE == kStats && isR) {          // A(i, k) = G[k][i]: two 64-wide boxes along i
+          tc::tma_load_3d(dst, mA, &full[s], i0, k0, pa * args.nblk + blk);
+          tc::tma_load_3d(dst + kBoxBytes / 2, mA, &full[s], i0 + 64, k0, pa * args.nblk + blk);
+        } else if (MODE == kApplyP) {         // A = L^{-1/p} planes
+          tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nmat + 2 * blk);
+        } else {                              // A = G rows
+          tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nblk + blk);
+        }
+      }
+      for (int pb = 0; pb < nB; ++pb) {
+        uint8_t* dst = st + (nA + pb) * kBoxBytes;
+        if (MODE == kStats && isR) {
+          tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
+          tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
+        } else if (MODE == kStats) {
+          tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nblk + blk);
+        } else if (MODE == kApplyY) {         // B(k, j) = R^{-1/p}[j][k] (symmetric)
+          tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nmat + 2 * blk + 1);
+        } else {                              // B(k, j) = Y[k][j], MN-major
+          tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
+          tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idesc = tc::idesc_bf16(kTM, kTM, a_mn, b_mn);
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % ST;
+      if (!tc::mbar_wait(&full[s], (kt / ST) & 1)) {
+        *abort_flag = 1;
+        atomicExch(args.err, tc::kErrTimeout);
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t st = tc::smem_u32(smem + s * stage_bytes);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        for (int q = 0; q < npass; ++q) {
+          const int pa = (pas >> (2 * q)) & 3;
+          const int pb = (pbs >> (2 * q)) & 3;
+          const uint32_t sa = st + pa * kBoxBytes;
+          const uint32_t sb = st + (nA + pb) * kBoxBytes;
+          const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
+                                   : tc::smem_desc(sa + kk * 32, 16, 1024);
+          const uint64_t db = b_mn ? tc::smem_desc(sb + kk * 2048, 8192, 1024)
+                                   : tc::smem_desc(sb + kk * 32, 16, 1024);
+          tc::mma_bf16(tmem, da, db, idesc, (kt | kk | q) != 0);
+        }
+      }
+      tc::mma_commit(&empty[s]);
+    }
+    tc::mma_commit(accum);
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: TMEM -> registers -> global ----------------
+  const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(accum, 0) && !*abort_flag);
+  tc::fence_after_sync();
+  const int r = i0 + warp * 32 + lane;         // output row owned by this thread
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  if (ok) {
+    if (MODE == kStats) {
+      float* C = args.stats + (size_t)(2 * blk + isR) * S * S;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tc::tmem_ld32(trow + c * 32, v);
+        const int cb = j0 + c * 32;
+        if (r < S && cb < S) {
+          float4* row = reinterpret_cast<float4*>(C + (size_t)r * S + cb);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 o = row[q];
+            o.x = fmaf(args.beta2, o.x, v[4 * q + 0]);
+            o.y = fmaf(args.beta2, o.y, v[4 * q + 1]);
+            o.z = fmaf(args.beta2, o.z, v[4 * q + 2]);
+            o.w = fmaf(args.beta2, o.w, v[4 * q + 3]);
+            row[q] = o;
+          }
+        }
+      }
+    } else if (MODE == kApplyY) {
+      uint16_t* yh = args.y + (size_t)blk * S * S;
+      uint16_t* yl = args.y + (size_t)(args.nblk + blk) * S * S;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tc::tmem_ld32(trow + c * 32, v);
+        const int cb = j0 + c * 32;
+        if (r < S && cb < S) {
+          uint32_t hw[16], lw[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const uint16_t h0 = tc::bf16_bits_rn(v[2 * q]), h1 = tc::bf16_bits_rn(v[2 * q + 1]);
+            const uint16_t l0 = tc::bf16_bits_rn(v[2 * q] - tc::bf16_to_f(h0));
+            const uint16_t l1 = tc::bf16_bits_rn(v[2 * q + 1] - tc::bf16_to_f(h1));
+            hw[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            lw[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+          }
+          uint4* dh = reinterpret_cast<uint4*>(yh + (size_t)r * S + cb);
+          uint4* dl = reinterpret_cast<uint4*>(yl + (size_t)r * S + cb);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            dh[q] = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+            dl[q] = make_uint4(lw[4 * q], lw[4 * q + 1], lw[4 * q + 2], lw[4 * q + 3]);
+          }
+        }
+      }
+    } else {
+      double ss = 0.0;
+      float* Pp = args.P + args.params[bd.param].offset;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tc::tmem_ld32(trow + c * 32, v);
+        const int cb = j0 + c * 32;
+        if (r < bd.m) {
+          float* dst = Pp + (bd.r0 + r) * bd.ld + bd.c0 + cb;
+          if (cb + 32 <= bd.n && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ss += (double)v[e] * v[e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (cb + e < bd.n) {
+                dst[e] = v[e];
+                ss += (double)v[e] * v[e];
+              }
+            }
+          }
+        }
+      }
+      ss = warp_sum(ss);
+      if (lane == 0 && ss != 0.0) atomicAdd(&args.p2[bd.param], ss);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
+// K1: gradients -> blocked, zero-padded bf16 planes.  grid: x = 2048-element
+// run of the S x S slot, y = block; each thread handles 8 consecutive columns.
+__global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict__ blocks,
+                                                     const void* const* __restrict__ gptr, int bf16,
+                                                     int* __restrict__ flags, int S, int nblk,
+                                                     uint16_t* __restrict__ out) {
+  const BlockDesc bd = blocks[blockIdx.y];
+  if (flags[bd.param]) return;
+  const int64_t e0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (e0 >= (int64_t)S * S) return;
+  const int i = (int)(e0 / S), j = (int)(e0 % S);
+  uint32_t hw[4] = {0, 0, 0, 0}, mw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
+  const void* g = gptr[bd.param];
+  const int64_t base = (bd.r0 + i) * bd.ld + bd.c0;
+  int bad = 0;
+  if (i < bd.m) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int jj = j + q;
+      if (jj < bd.n) {
+        uint16_t h, m = 0, l = 0;
+        if (bf16) {
+          h = __ldg(reinterpret_cast<const uint16_t*>(g) + base + jj);
+          bad |= (h & 0x7F80) == 0x7F80;
+        } else {
+          const float x = __ldg(reinterpret_cast<const float*>(g) + base + jj);
+          bad |= !isfinite(x);
+          h = tc::bf16_bits_rn(x);
+          const float r1 = x - tc::bf16_to_f(h);        // exact
+          m = tc::bf16_bits_rn(r1);
+          l = tc::bf16_bits_rn(r1 - tc::bf16_to_f(m));  // exact remainder, rounded
+        }
+        hw[q >> 1] |= (uint32_t)h << (16 * (q & 1));
+        mw[q >> 1] |= (uint32_t)m << (16 * (q & 1));
+        lw[q >> 1] |= (uint32_t)l << (16 * (q & 1));
+      }
+    }
+  }
+  if (bad) atomicOr(&flags[bd.param], 1);
+  const size_t slot = (size_t)S * S;
+  *reinterpret_cast<uint4*>(out + blockIdx.y * slot + e0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  if (!bf16) {
+    *reinterpret_cast<uint4*>(out + (nblk + blockIdx.y) * slot + e0) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+    *reinterpret_cast<uint4*>(out + (2 * (size_t)nblk + blockIdx.y) * slot + e0) =
+        make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+// roots (fp32, [nmat][S][S]) -> bf16 planes hi [nmat] then lo [nmat]
+__global__ void split_kernel(const float* __restrict__ x, int64_t n, uint16_t* __restrict__ out) {
+  for (int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; e < n;
+       e += (int64_t)gridDim.x * blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(x + e);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    uint16_t h[4], l[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      h[q] = tc::bf16_bits_rn(f[q]);
+      l[q] = tc::bf16_bits_rn(f[q] - tc::bf16_to_f(h[q]));
+    }
+    *reinterpret_cast<uint2*>(out + e) =
+        make_uint2((uint32_t)h[0] | ((uint32_t)h[1] << 16), (uint32_t)h[2] | ((uint32_t)h[3] << 16));
+    *reinterpret_cast<uint2*>(out + n + e) =
+        make_uint2((uint32_t)l[0] | ((uint32_t)l[1] << 16), (uint32_t)l[2] | ((uint32_t)l[3] << 16));
+  }
+}
+
+int stage_count(int stage_bytes) { return stage_bytes <= 3 * kBoxBytes ? 3 : 2; }
+
+size_t smem_bytes(int nA, int nB) {
+  const int sb = (nA + nB) * kBoxBytes;
+  return (size_t)stage_count(sb) * sb + 1024 + 256;
+}
+
+template <int MODE>
+cudaError_t launch_mode(dim3 grid, size_t smem, const TcMaps& maps, const TcArgs& a, cudaStream_t s) {
+  static bool configured = false;   // per process; the attribute is per function
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         200 * 1024);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  tc_gemm_kernel<MODE><<<grid, 128, smem, s>>>(maps.gk, maps.gmn, maps.rk, maps.ymn, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
+                          int* flags, int S, uint16_t* out, cudaStream_t s) {
+  if (nblk <= 0) return cudaSuccess;
+  dim3 grid((unsigned)(((int64_t)S * S / 8 + 255) / 256), nblk);
+  gather_kernel<<<grid, 256, 0, s>>>(blocks, gptr, bf16, flags, S, nblk, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split(const float* x, int64_t n, uint16_t* out, cudaStream_t s) {
+  split_kernel<<<1184, 256, 0, s>>>(x, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
+                            int nmat, int S, int planes_g, float beta2, float* stats, int* err,
+                            cudaStream_t s) {
+  if (nblk <= 0) return cudaSuccess;
+  TcArgs a{};
+  a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
+  a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err;
+  const int T = (S + kTM - 1) / kTM;
+  return launch_mode<kStats>(dim3(T * (T + 1) / 2, nblk, 2), smem_bytes(planes_g, planes_g), maps, a, s);
+}
+
+cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
+                              int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s) {
+  if (nblk <= 0) return cudaSuccess;
+  TcArgs a{};
+  a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
+  a.planes_g = planes_g; a.y = y; a.err = err;
+  const int T = (S + kTM - 1) / kTM;
+  return launch_mode<kApplyY>(dim3(T * T, nblk), smem_bytes(planes_g == 1 ? 1 : 2, 2), maps, a, s);
+}
+
+cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const ParamDesc* params,
+                              const int* flags, int nblk, int nmat, int S, float* P, double* p2,
+                              int* err, cudaStream_t s) {
+  if (nblk <= 0) return cudaSuccess;
+  TcArgs a{};
+  a.blocks = blocks; a.params = params; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
+  a.planes_g = 2; a.P = P; a.p2 = p2; a.err = err;
+  const int T = (S + kTM - 1) / kTM;
+  return launch_mode<kApplyP>(dim3(T * T, nblk), smem_bytes(2, 2), maps, a, s);
+}
+
+}  // namespace shampoo
