@@ -205,6 +205,8 @@ cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
     if ((e = dalloc(ctx, b, mat)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.cinv, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.ridge, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.sched, (size_t)chunk * kSched)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.nsched, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.resid, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.prev, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.worse, chunk)) != cudaSuccess) return e;
@@ -251,6 +253,8 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
         launch_newton_bound(A, a_stride, lda, upper, d, nm, eps, attempt, w, st);
       });
       run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, upper, d, nm, S, w, st); });
+      run(pr, "newton_lanczos", st, [&] { launch_newton_lanczos(d, nm, S, w, st); });
+      run(pr, "newton_t0", st, [&] { launch_newton_t0(d, nm, S, w, st); });
       run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
       CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
       CK(cudaEventRecord(ev[0], st));

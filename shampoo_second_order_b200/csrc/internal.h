@@ -35,6 +35,7 @@ struct ParamDesc {
 };
 
 constexpr int kChunk = 16384;   // elements per elementwise chunk
+constexpr int kSched = 32;      // longest Newton scaling schedule
 constexpr int kTile = 64;       // tile side of every matrix kernel
 
 // Per-matrix bookkeeping of the Newton root iteration.
@@ -88,6 +89,8 @@ struct NewtonWork {
   double* T4;
   double* cinv;                 // [nmat] c^{-1}
   double* ridge;                // [nmat] ridge added to A (eps, raised on a retry)
+  double* sched;                // [nmat][kSched] scaling s_k of the first steps
+  int* nsched;                  // [nmat] number of scaled steps
   unsigned long long* resid;    // [nmat] max|M-I| as ordered bits
   double* prev;                 // [nmat] previous residual
   int* worse;                   // [nmat]
@@ -107,6 +110,9 @@ void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, c
                          int nm, float eps, int attempt, NewtonWork w, cudaStream_t s);
 void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
                         int nm, int S, NewtonWork w, cudaStream_t s);
+// Lanczos estimate of M0's spectrum and the scaling schedule, then T0.
+void launch_newton_lanczos(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
+void launch_newton_t0(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
 // one Newton step: A (X T and T T), B (T2 T2, p = 4 only), C (T^p M,
 // residual, next T); check k: convergence test of M_k
 void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);

@@ -1,16 +1,31 @@
 // Batched inverse p-th roots by the coupled Newton iteration in float64
 // (transcript segment 12: the root must be taken in double precision; this
-// is the coupled Newton iteration it names, Guo & Higham 2006):
+// is the coupled Newton iteration it names, Guo & Higham 2006), with a scalar
+// scaling of the first steps:
 //
 //   c^p >= lambda_max(A + eps I),  X0 = c^{-1} I,  M0 = (A + eps I) / c^p
-//   T = ((p+1) I - M) / p,  X <- X T,  M <- T^p M,   until max|M - I| <= tol
+//   step k:  T = ((p+1) I - s_k M) / p,  X <- s_k^{1/p} X T,  M <- s_k T^p M
+//   until max|M - I| <= tol.
+//
+// Scaling X by mu and M by mu^p keeps the coupling M = X^p (A + eps I), so
+// every s_k > 0 leaves the limit unchanged.  Each eigenvalue m of M moves by
+// the scalar map m -> s m ((p+1 - s m)/p)^p, which for s = 1 (plain Newton)
+// only multiplies small eigenvalues by ((p+1)/p)^p per step.  A short Lanczos
+// run on M0 estimates its extreme eigenvalues [l, u]; s_k is then chosen so
+// that the ends of the current interval land on the same value (equal
+// oscillation), which roughly halves the steps for spread spectra.  s_k is
+// capped at 0.98 (p+1) so that the true top eigenvalue (<= 1 by the choice
+// of c) stays inside the map's convergence region whatever the estimate;
+// a poor estimate costs steps, never the limit.  Once the tracked interval
+// sits above 0.7 the plain iteration finishes quadratically.
 //
 // Every matrix the iteration touches is a polynomial in A, so all of them are
 // symmetric and commute: each product is computed on the upper-triangular
 // 64 x 64 tiles only and written to both (i, j) and (j, i).  The products run
 // on the float64 tensor-core MMA (mma.sync m8n8k4 .f64).  A ragged statistic
 // sits in the top-left corner of its S x S slot; the padding is set to the
-// identity in M (so T = I there) and never mixes with the valid corner.
+// identity in M0, never mixes with the valid corner, and is left out of the
+// residual.
 #include <float.h>
 
 #include "common.cuh"
@@ -183,8 +198,8 @@ __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restri
   }
 }
 
-// grid: x = row of the S x S slot, y = matrix.  Writes X0, M0, T0 into the
-// parity-0 buffers and folds max|M0 - I| into the residual.
+// grid: x = row of the S x S slot, y = matrix.  Writes X0, M0 into the
+// parity-0 buffers and folds max|M0 - I| (valid corner) into the residual.
 __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restrict__ A,
                                                           int64_t a_stride, int lda, int upper,
                                                           const NewtonMat* __restrict__ mats,
@@ -199,11 +214,11 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
   const double inv_cp = 1.0 / cpow[m];
   const double rd = w.ridge[m];
   const double ci = w.cinv[m];
-  const double pinv = 1.0 / mt.p;
   double dev = 0.0;
   for (int c = threadIdx.x; c < S; c += blockDim.x) {
     double v;
-    if (r < mt.size && c < mt.size) {
+    const bool valid = r < mt.size && c < mt.size;
+    if (valid) {
       v = (double)sym_at(a, lda, upper, r, c);
       if (r == c) v += rd;
       v *= inv_cp;
@@ -212,14 +227,173 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
     }
     const double d = (r == c) ? 1.0 : 0.0;
     w.M[0][off + c] = v;
-    w.T[off + c] = ((mt.p + 1) * d - v) * pinv;
     w.X[0][off + c] = (r == c) ? ci : 0.0;
-    double e = fabs(v - d);
+    double e = valid ? fabs(v - d) : 0.0;
     if (!(e <= DBL_MAX)) e = INFINITY;
     dev = fmax(dev, e);
   }
   dev = block_max(dev, red);
   if (threadIdx.x == 0) atomicMax(&w.resid[m], dbl_bits(dev));
+}
+
+// ---------------------------------------------------------------------------
+// Scaling schedule
+// ---------------------------------------------------------------------------
+constexpr int kLanczos = 16;
+
+__device__ __forceinline__ double newton_map(double m, int p) {
+  const double t = (p + 1 - m) / p;
+  const double t2 = t * t;
+  return m * (p == 4 ? t2 * t2 : t2);
+}
+
+// Number of eigenvalues of the symmetric tridiagonal (a, b) below x.
+__device__ int sturm_count(const double* a, const double* b, int k, double x) {
+  int cnt = 0;
+  double d = a[0] - x;
+  if (d < 0) ++cnt;
+  for (int i = 1; i < k; ++i) {
+    const double dd = (d == 0.0) ? 1e-300 : d;
+    d = a[i] - x - b[i - 1] * b[i - 1] / dd;
+    if (d < 0) ++cnt;
+  }
+  return cnt;
+}
+
+// Smallest (which = 1) or largest (which = k) eigenvalue of the tridiagonal.
+__device__ double tridiag_eig(const double* a, const double* b, int k, int which) {
+  double lo = a[0], hi = a[0];
+  for (int i = 0; i < k; ++i) {
+    const double r = (i > 0 ? fabs(b[i - 1]) : 0.0) + (i + 1 < k ? fabs(b[i]) : 0.0);
+    lo = fmin(lo, a[i] - r);
+    hi = fmax(hi, a[i] + r);
+  }
+  for (int it = 0; it < 100; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (sturm_count(a, b, k, mid) >= which) hi = mid;
+    else lo = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// One CTA per matrix: kLanczos Lanczos steps on the valid corner of M0
+// (float64, no reorthogonalisation: only the extreme Ritz values are used),
+// their extreme eigenvalues by Sturm bisection, and the schedule s_k.
+__global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __restrict__ mats, int S,
+                                                             NewtonWork w) {
+  __shared__ double v[1024], vp[1024], wv[1024];
+  __shared__ double al[kLanczos], be[kLanczos];
+  __shared__ double red[16];
+  __shared__ double bcast;
+  const int m = blockIdx.x;
+  const NewtonMat mt = mats[m];
+  const int n = mt.size, p = mt.p;
+  const double* M = w.M[0] + (size_t)m * S * S;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // start vector: a fixed pseudo-random +-1 pattern (hash of the index)
+  double ss = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    uint32_t h = (uint32_t)i * 2654435761u;
+    h ^= h >> 15;
+    const double x = (h & 1u) ? 1.0 : -1.0;
+    v[i] = x;
+    vp[i] = 0.0;
+    ss += x * x;
+  }
+  ss = block_sum(ss, red);
+  if (threadIdx.x == 0) bcast = 1.0 / sqrt(ss);
+  __syncthreads();
+  const double inv0 = bcast;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) v[i] *= inv0;
+  __syncthreads();
+  double beta = 0.0;
+  int kk = 0;
+  for (int j = 0; j < kLanczos && j < n; ++j) {
+    for (int r = warp; r < n; r += nw) {
+      const double* row = M + (size_t)r * S;
+      double d = 0.0;
+      for (int c = lane; c < n; c += 32) d += row[c] * v[c];
+      d = warp_sum(d);
+      if (lane == 0) wv[r] = d - beta * vp[r];
+    }
+    __syncthreads();
+    double a = 0.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) a += v[i] * wv[i];
+    a = block_sum(a, red);
+    if (threadIdx.x == 0) bcast = a;
+    __syncthreads();
+    a = bcast;
+    double b2 = 0.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const double x = wv[i] - a * v[i];
+      wv[i] = x;
+      b2 += x * x;
+    }
+    b2 = block_sum(b2, red);
+    if (threadIdx.x == 0) bcast = sqrt(b2);
+    __syncthreads();
+    const double b = bcast;
+    if (threadIdx.x == 0) {
+      al[j] = a;
+      be[j] = b;
+    }
+    kk = j + 1;
+    if (!(b > 1e-13 * fabs(a)) || !(b <= DBL_MAX)) break;   // invariant subspace (or garbage)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      vp[i] = v[i];
+      v[i] = wv[i] / b;
+    }
+    beta = b;
+    __syncthreads();
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  // interval estimate, kept inside what is guaranteed: [ridge / c^p, 1]
+  const double lo_g = w.ridge[m] / w.T2[m];   // T2 holds c^p until the first step
+  double l = tridiag_eig(al, be, kk, 1), u = tridiag_eig(al, be, kk, kk);
+  int ns = 0;
+  double* sch = w.sched + (size_t)m * kSched;
+  if (l <= DBL_MAX && u <= DBL_MAX && l > 0.0) {
+    u = fmin(1.0, u * 1.02);
+    l = fmin(fmax(l, lo_g), u);
+    const double cap = 0.98 * (p + 1);
+    while (ns < kSched && l < 0.7) {
+      // s in [1/u, min((p+1)/u, cap)] with map(s l) = map(s u)
+      double a = 1.0 / u, b = fmin((p + 1) / u, cap), s;
+      if (newton_map(b * l, p) <= newton_map(b * u, p)) {
+        s = b;
+      } else {
+        for (int it = 0; it < 80; ++it) {
+          const double mid = 0.5 * (a + b);
+          if (newton_map(mid * l, p) < newton_map(mid * u, p)) a = mid;
+          else b = mid;
+        }
+        s = 0.5 * (a + b);
+      }
+      const double x = newton_map(s * l, p), y = newton_map(s * u, p);
+      const double nl = fmin(x, y);
+      const double nu = (s * l <= 1.0 && s * u >= 1.0) ? 1.0 : fmax(x, y);
+      l = nl;
+      u = fmax(nu, nl);
+      sch[ns++] = s;
+    }
+  }
+  w.nsched[m] = ns;
+}
+
+__device__ __forceinline__ double sched_at(const NewtonWork& w, int m, int k) {
+  return k < w.nsched[m] ? w.sched[(size_t)m * kSched + k] : 1.0;
+}
+
+// T0 = ((p+1) I - s_0 M0) / p.  grid: x = row, y = matrix.
+__global__ void __launch_bounds__(256) newton_t0_kernel(const NewtonMat* __restrict__ mats, int S,
+                                                        NewtonWork w) {
+  const int m = blockIdx.y, r = blockIdx.x;
+  const int p = mats[m].p;
+  const double s0 = sched_at(w, m, 0), pinv = 1.0 / p;
+  const size_t off = (size_t)m * S * S + (size_t)r * S;
+  for (int c = threadIdx.x; c < S; c += blockDim.x)
+    w.T[off + c] = ((p + 1) * (r == c ? 1.0 : 0.0) - s0 * w.M[0][off + c]) * pinv;
 }
 
 // ---------------------------------------------------------------------------
@@ -229,7 +403,7 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
 //   M_next = T^p M, residual, T <- ((p+1) I - M_next)/p  (launch C)
 // grid: x = upper-triangular tile, y = matrix, z = job.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kNewtonThreads) newton_step_a_kernel(
+__global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
     const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
   __shared__ NewtonSmem sm;
   const int m = blockIdx.y;
@@ -243,10 +417,23 @@ __global__ void __launch_bounds__(kNewtonThreads) newton_step_a_kernel(
   double* C = blockIdx.z == 0 ? w.X[(it + 1) & 1] + base : w.T2 + base;
   double acc[4][4][2] = {};
   dmma_tile(A, Tm, S, ti * kTile, tj * kTile, acc, sm);
+  if (blockIdx.z == 0) {   // X_next = s_k^{1/p} X T
+    const double sk = sched_at(w, m, it);
+    if (sk != 1.0) {
+      const double mu = pow(sk, 1.0 / mats[m].p);
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+          acc[mi][ni][0] *= mu;
+          acc[mi][ni][1] *= mu;
+        }
+    }
+  }
   store_sym(C, S, ti * kTile, tj * kTile, acc);
 }
 
-__global__ void __launch_bounds__(kNewtonThreads) newton_step_b_kernel(
+__global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_b_kernel(
     const NewtonMat* __restrict__ mats, int S, NewtonWork w) {
   __shared__ NewtonSmem sm;
   const int m = blockIdx.y;
@@ -260,7 +447,7 @@ __global__ void __launch_bounds__(kNewtonThreads) newton_step_b_kernel(
   store_sym(w.T4 + base, S, ti * kTile, tj * kTile, acc);
 }
 
-__global__ void __launch_bounds__(kNewtonThreads) newton_step_c_kernel(
+__global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
     const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
   __shared__ NewtonSmem sm;
   __shared__ double red[kNewtonThreads / 32];
@@ -275,11 +462,21 @@ __global__ void __launch_bounds__(kNewtonThreads) newton_step_c_kernel(
   double acc[4][4][2] = {};
   const int i0 = ti * kTile, j0 = tj * kTile;
   dmma_tile(Tp, w.M[it & 1] + base, S, i0, j0, acc, sm);
+  // M_next = s_k T^p M
+  const double sk = sched_at(w, m, it), sn = sched_at(w, m, it + 1);
+#pragma unroll
+  for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni) {
+      acc[mi][ni][0] *= sk;
+      acc[mi][ni][1] *= sk;
+    }
   store_sym(w.M[(it + 1) & 1] + base, S, i0, j0, acc);
-  // residual and the next T from the same accumulators
+  // residual (valid corner) and the next T = ((p+1) I - s_{k+1} M_next) / p
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int wm = warp >> 1, wn = warp & 1;
+  const int n = mats[m].size;
   const double pinv = 1.0 / p;
   double dev = 0.0;
 #pragma unroll
@@ -291,10 +488,10 @@ __global__ void __launch_bounds__(kNewtonThreads) newton_step_c_kernel(
         const int r = i0 + wm * 32 + mi * 8 + g;
         const int c = j0 + wn * 32 + ni * 8 + 2 * t + e;
         const double d = (r == c) ? 1.0 : 0.0;
-        double x = fabs(acc[mi][ni][e] - d);
+        double x = (r < n && c < n) ? fabs(acc[mi][ni][e] - d) : 0.0;
         if (!(x <= DBL_MAX)) x = INFINITY;
         dev = fmax(dev, x);
-        acc[mi][ni][e] = ((p + 1) * d - acc[mi][ni][e]) * pinv;
+        acc[mi][ni][e] = ((p + 1) * d - sn * acc[mi][ni][e]) * pinv;
       }
   store_sym(w.T + base, S, i0, j0, acc);
   dev = block_max(dev, red);
@@ -319,7 +516,7 @@ __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, Ne
       st = kConverged;
     } else if (k >= max_iters) {
       st = kFailed;
-    } else {
+    } else if (k >= w.nsched[m]) {   // the scaled steps may raise the residual
       const int wo = (r >= w.prev[m]) ? w.worse[m] + 1 : 0;
       w.worse[m] = wo;
       w.prev[m] = r;
@@ -340,6 +537,7 @@ __global__ void newton_reset_kernel(int nm, NewtonWork w) {
     w.prev[m] = INFINITY;
     w.worse[m] = 0;
     w.iters[m] = 0;
+    w.nsched[m] = 0;
   }
 }
 
@@ -388,6 +586,14 @@ void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, c
 void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
                         int nm, int S, NewtonWork w, cudaStream_t s) {
   newton_init_kernel<<<dim3(S, nm), 256, 0, s>>>(A, a_stride, lda, upper, mats, S, w, w.T2);
+}
+
+void launch_newton_lanczos(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {
+  newton_lanczos_kernel<<<nm, 512, 0, s>>>(mats, S, w);
+}
+
+void launch_newton_t0(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {
+  newton_t0_kernel<<<dim3(S, nm), 256, 0, s>>>(mats, S, w);
 }
 
 static int num_tri(int S) {

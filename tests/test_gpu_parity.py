@@ -255,3 +255,21 @@ def test_nan_statistic_fails_root_and_keeps_previous():
     iters = iters.cpu().numpy()
     assert iters[0] >= 0 and iters[1] < 0
     assert np.allclose(X[0].cpu().numpy(), (2 + 1e-6) ** -0.25 * np.eye(64), rtol=1e-6)
+
+
+def test_scaled_newton_takes_fewer_steps_than_plain():
+    """The Lanczos-scaled iteration reaches the same root (checked above) in
+    fewer steps than the plain coupled Newton iteration needs on the same
+    matrices (the oracle's CPU copy of the pages' root route)."""
+    from oracle import coupled_newton_inverse_root
+    from shampoo_second_order_b200 import batched_inverse_root
+    A, _ = wl.spd_batch(8, 256, seed=31, log10_kappa=(2.0, 6.0))
+    A32 = A.astype(np.float32)
+    X, iters = batched_inverse_root(torch.from_numpy(A32).cuda(), 4, 1e-6)
+    iters = iters.cpu().numpy()
+    X = X.cpu().numpy()
+    for i in range(8):
+        _, k_plain, ok = coupled_newton_inverse_root(A32[i].astype(np.float64), 1e-6, 4)
+        assert ok and 0 < iters[i] < k_plain, (i, iters[i], k_plain)
+        ref = inverse_root(A32[i].astype(np.float64), 1e-6, 4)
+        assert rel(X[i], ref) <= ROOT_TOL
