@@ -99,6 +99,21 @@ def numel(cfg):
     return wl.count_params(cfg["shapes"])
 
 
+def max_over_ranks(ms, dist, device):
+    """The job time: the largest per-rank device time (one all-reduce)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank, world, job_ms):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (job_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
@@ -448,16 +463,11 @@ def main():
     clk = clocks.stop()
     prof = opt.profile_read()
     opt.profile_enable(False)
-    total_ms = sum(s.elapsed_time(e) for s, e in ev)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        dist.barrier()
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), dist if world > 1 else None, dev)
     launches = sum(v[0] for v in prof.values())
 
     flops_rank = args.steps * (stats_flops(cfg) + apply_flops(cfg)) + newton_flops(cfg, iters_sum)
-    value = world * flops_rank / (total_ms * 1e-3) / 1e12
+    value = job_tflops(flops_rank, world, total_ms)
 
     # ---- e2e: host buffers through the public API ----
     e2e = None
@@ -480,12 +490,8 @@ def main():
                     h.copy_(d, non_blocking=True)
                 eve[j][1].record(stream)
         stream.synchronize()
-        e2e_ms = sum(s.elapsed_time(e) for s, e in eve)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * flops_rank / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in eve), dist if world > 1 else None, dev)
+        e2e = {"value": job_tflops(flops_rank, world, e2e_ms), "unit": UNIT,
                "ms_per_step": e2e_ms / args.steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak)
