@@ -233,6 +233,35 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
                                             int max_iters, int32_t* iters,
                                             void* stream);
 
+/*
+ * shampoo_batched_inverse_root_noalloc -- shampoo_batched_inverse_root for
+ * callers that cannot allocate device memory.  (The paper has no counterpart:
+ * this is a deployment variant of the same root computation.)
+ *
+ * Who needs it: code whose device memory is owned by a framework's pooling
+ * allocator (a raw cudaMalloc there fragments the pool or fails once the pool
+ * has reserved the GPU), code on a path where an allocation's implicit
+ * synchronisation is not acceptable, and hosts that forbid allocating after
+ * start-up.  This call allocates nothing -- no cudaMalloc, cudaFree, pinned
+ * host memory, CUDA events or library allocator.  Its float64 work space is
+ * one 64 MiB array compiled into the library, present on every GPU that loads
+ * the library until the process exits.
+ *
+ * Arguments, outputs and results are those of shampoo_batched_inverse_root
+ * (A, X and iters are caller-owned device memory).  Limits: n <= 1024; larger
+ * n is rejected with SHAMPOO_EINVAL and a message from shampoo_last_error(NULL).
+ * Any batch size is accepted; matrices are processed in chunks that fit the
+ * work space (7 n' x n' doubles each, n' = n rounded up to 64).
+ * Sharing: every call uses the same work space, so calls that overlap on the
+ * GPU (from other streams or host threads) race; serialise them.  The first
+ * call on a device looks up the work space's device address with that device
+ * current; make that first call before any stream capture.  Synchronises
+ * with the host while it runs.
+ */
+shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, float* X, int batch, int n,
+                                                    int p, float eps, double tol, int max_iters,
+                                                    int32_t* iters, void* stream);
+
 /* Library version, "MAJOR.MINOR.PATCH". */
 const char* shampoo_version(void);
 

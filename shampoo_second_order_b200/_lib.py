@@ -39,6 +39,8 @@ SIGNATURES = {
     "shampoo_destroy": (None, [_P]),
     "shampoo_batched_inverse_root": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_float,
                                                C.c_double, C.c_int, _P, _P]),
+    "shampoo_batched_inverse_root_noalloc": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_float,
+                                                       C.c_double, C.c_int, _P, _P]),
     "shampoo_version": (C.c_char_p, []),
 }
 
@@ -175,6 +177,15 @@ def shampoo_batched_inverse_root(A_ptr, X_ptr, batch, n, p, eps, tol, max_iters,
                                             int(batch), int(n), int(p), float(eps), float(tol),
                                             int(max_iters), C.c_void_p(int(iters_ptr)),
                                             C.c_void_p(int(stream)))
+    return _check(st, None, allow=(ENOTCONVERGED,))
+
+
+def shampoo_batched_inverse_root_noalloc(A_ptr, X_ptr, batch, n, p, eps, tol, max_iters, iters_ptr=0,
+                                         stream=0):
+    st = lib().shampoo_batched_inverse_root_noalloc(C.c_void_p(int(A_ptr)), C.c_void_p(int(X_ptr)),
+                                                    int(batch), int(n), int(p), float(eps), float(tol),
+                                                    int(max_iters), C.c_void_p(int(iters_ptr)),
+                                                    C.c_void_p(int(stream)))
     return _check(st, None, allow=(ENOTCONVERGED,))
 
 

@@ -373,6 +373,12 @@ shampoo_status gather(shampoo_ctx* ctx, const void* const* grads, bool force) {
 
 }  // namespace
 
+namespace shampoo {
+// The error text shampoo_last_error(NULL) returns, for entry points without a
+// context that live in other files.
+void set_global_error(const std::string& msg) { g_create_err = msg; }
+}  // namespace shampoo
+
 extern "C" {
 
 const char* shampoo_version(void) { return "0.1.0"; }
