@@ -208,6 +208,7 @@ cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
   if ((e = dalloc(ctx, &w.sched, (size_t)chunk * kSched)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.nsched, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.resid, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.fro2, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.prev, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.worse, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.iters, chunk)) != cudaSuccess) return e;

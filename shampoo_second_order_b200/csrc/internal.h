@@ -92,11 +92,13 @@ struct NewtonWork {
   double* sched;                // [nmat][kSched] scaling s_k of the first steps
   int* nsched;                  // [nmat] number of scaled steps
   unsigned long long* resid;    // [nmat] max|M-I| as ordered bits
+  double* fro2;                 // [nmat] ||M-I||_F^2 of the valid corner
   double* prev;                 // [nmat] previous residual
   int* worse;                   // [nmat]
   int* active;                  // [nmat]
   int* iters;                   // [nmat] iterations done
-  int* state;                   // [nmat] 0 running, 1 converged, 2 failed, 3 diverged
+  int* state;                   // [nmat] 0 running, 1 converged, 2 failed, 3 diverged,
+                                //        4 one X-only step left
   int* count;                   // [1] matrices still active after a check
 };
 // Set up X0, M0, T0 for `nm` matrices read from `A` (float32, slot-strided

@@ -17,7 +17,10 @@
 // capped at 0.98 (p+1) so that the true top eigenvalue (<= 1 by the choice
 // of c) stays inside the map's convergence region whatever the estimate;
 // a poor estimate costs steps, never the limit.  Once the tracked interval
-// sits above 0.7 the plain iteration finishes quadratically.
+// sits above 0.7 the plain iteration finishes quadratically: near 1 the map
+// sends 1 - m to (p+1)/(2p) (1 - m)^2 + O((1 - m)^3), so when ||M - I||_F = f
+// bounds every |1 - m| and 0.75 f^2 (1 + f) <= tol / 2, the next step's
+// residual is certainly below tol and that step computes X <- X T alone.
 //
 // Every matrix the iteration touches is a polynomial in A, so all of them are
 // symmetric and commute: each product is computed on the upper-triangular
@@ -39,7 +42,7 @@ constexpr int kBK = 16;
 constexpr int kAStride = kBK + 4;     // doubles; 4 mod 16 keeps fragment loads conflict-free
 constexpr int kBStride = kTile + 4;
 
-enum : int { kRunning = 0, kConverged = 1, kFailed = 2, kDiverged = 3 };
+enum : int { kRunning = 0, kConverged = 1, kFailed = 2, kDiverged = 3, kFinal = 4 };
 
 __device__ __forceinline__ unsigned long long dbl_bits(double v) {
   return static_cast<unsigned long long>(__double_as_longlong(v));
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
 // ---------------------------------------------------------------------------
 // Scaling schedule
 // ---------------------------------------------------------------------------
-constexpr int kLanczos = 16;
+constexpr int kLanczos = 12;
 
 __device__ __forceinline__ double newton_map(double m, int p) {
   const double t = (p + 1 - m) / p;
@@ -305,15 +308,23 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
   __syncthreads();
   const double inv0 = bcast;
   for (int i = threadIdx.x; i < n; i += blockDim.x) v[i] *= inv0;
+  if (threadIdx.x == 0 && (n & 1)) v[n] = 0.0;   // pad for the pairwise row loads
   __syncthreads();
+  const int n2 = (n + 1) >> 1;
   double beta = 0.0;
   int kk = 0;
   for (int j = 0; j < kLanczos && j < n; ++j) {
     for (int r = warp; r < n; r += nw) {
-      const double* row = M + (size_t)r * S;
-      double d = 0.0;
-      for (int c = lane; c < n; c += 32) d += row[c] * v[c];
-      d = warp_sum(d);
+      // 16-byte loads; column n of an odd-sized corner is padding (0 here)
+      const double2* row = reinterpret_cast<const double2*>(M + (size_t)r * S);
+      double d0 = 0.0, d1 = 0.0;
+#pragma unroll 4
+      for (int c2 = lane; c2 < n2; c2 += 32) {
+        const double2 x = row[c2];
+        d0 = fma(x.x, v[2 * c2], d0);
+        d1 = fma(x.y, v[2 * c2 + 1], d1);
+      }
+      const double d = warp_sum(d0 + d1);
       if (lane == 0) wv[r] = d - beta * vp[r];
     }
     __syncthreads();
@@ -343,7 +354,7 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
       vp[i] = v[i];
       v[i] = wv[i] / b;
     }
-    beta = b;
+    beta = b;   // v[n] stays 0 for odd n
     __syncthreads();
   }
   __syncthreads();
@@ -407,7 +418,8 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
     const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
   __shared__ NewtonSmem sm;
   const int m = blockIdx.y;
-  if (w.state[m] != kRunning) return;
+  const int st = w.state[m];
+  if (st != kRunning && !(st == kFinal && blockIdx.z == 0)) return;
   const int T = S / kTile;
   int ti, tj;
   tri_tile(blockIdx.x, T, ti, tj);
@@ -478,7 +490,7 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
   const int wm = warp >> 1, wn = warp & 1;
   const int n = mats[m].size;
   const double pinv = 1.0 / p;
-  double dev = 0.0;
+  double dev = 0.0, f2 = 0.0;
 #pragma unroll
   for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
@@ -491,11 +503,17 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
         double x = (r < n && c < n) ? fabs(acc[mi][ni][e] - d) : 0.0;
         if (!(x <= DBL_MAX)) x = INFINITY;
         dev = fmax(dev, x);
+        // off-diagonal tiles stand for their mirror image too
+        f2 += (i0 == j0 ? 1.0 : 2.0) * x * x;
         acc[mi][ni][e] = ((p + 1) * d - sn * acc[mi][ni][e]) * pinv;
       }
   store_sym(w.T + base, S, i0, j0, acc);
   dev = block_max(dev, red);
-  if (threadIdx.x == 0) atomicMax(&w.resid[m], dbl_bits(dev));
+  f2 = block_sum(f2, red);
+  if (threadIdx.x == 0) {
+    atomicMax(&w.resid[m], dbl_bits(dev));
+    atomicAdd(&w.fro2[m], f2);
+  }
 }
 
 // Convergence test of M_k for every matrix (k = iterations done), in the
@@ -503,9 +521,16 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
 __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, NewtonWork w) {
   int alive = 0;
   for (int m = threadIdx.x; m < nm; m += blockDim.x) {
+    if (w.state[m] == kFinal) {   // its last step computed X alone
+      w.state[m] = kConverged;
+      w.iters[m] = k;
+      continue;
+    }
     if (w.state[m] != kRunning) continue;
     const double r = __longlong_as_double(static_cast<long long>(w.resid[m]));
+    const double f = sqrt(w.fro2[m]);
     w.resid[m] = 0ull;
+    w.fro2[m] = 0.0;
     w.iters[m] = k;
     // For a PSD A every eigenvalue of M stays in (0, 1], so max|M - I| < 1;
     // a residual above 1.5 means rounding made A + ridge I indefinite.
@@ -516,6 +541,8 @@ __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, Ne
       st = kConverged;
     } else if (k >= max_iters) {
       st = kFailed;
+    } else if (k >= w.nsched[m] && k > 0 && f <= 0.05 && 0.75 * f * f * (1.0 + f) <= 0.5 * tol) {
+      st = kFinal;   // one more step certainly lands below tol: compute X only
     } else if (k >= w.nsched[m]) {   // the scaled steps may raise the residual
       const int wo = (r >= w.prev[m]) ? w.worse[m] + 1 : 0;
       w.worse[m] = wo;
@@ -523,7 +550,7 @@ __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, Ne
       if (wo >= 5) st = kDiverged;
     }
     w.state[m] = st;
-    alive += (st == kRunning);
+    alive += (st == kRunning || st == kFinal);
   }
   // number of threads still holding a running matrix: zero iff none runs
   alive = __syncthreads_count(alive);
@@ -534,6 +561,7 @@ __global__ void newton_reset_kernel(int nm, NewtonWork w) {
   for (int m = threadIdx.x; m < nm; m += blockDim.x) {
     w.state[m] = kRunning;
     w.resid[m] = 0ull;
+    w.fro2[m] = 0.0;
     w.prev[m] = INFINITY;
     w.worse[m] = 0;
     w.iters[m] = 0;

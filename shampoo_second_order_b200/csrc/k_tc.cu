@@ -16,10 +16,13 @@
 // accuracy.  The apply products keep hi*hi + hi*lo + lo*hi of two-term
 // splits (relative error near 2^-16), well inside the step tolerance.
 //
-// One CTA computes one 128 x 128 output tile with 128 threads: lane 0 of
-// warp 0 issues TMA loads into a ring of shared-memory stages, lane 0 of warp
-// 1 issues the MMAs and releases stages through tcgen05.commit, and all four
-// warps then read the accumulator out of TMEM (warp w owns rows 32w..32w+31).
+// The GEMM kernel is persistent and warp-specialised: one CTA per SM walks
+// the 128 x 128 output tiles round-robin with 192 threads.  Lane 0 of warp 0
+// issues TMA loads into a ring of shared-memory stages, lane 0 of warp 1
+// issues the MMAs into one of two TMEM accumulators and releases stages with
+// tcgen05.commit, and warps 2-5 drain the other accumulator (warp w owns TMEM
+// lanes 32 (w % 4) ..), so the epilogue of one tile overlaps the main loop of
+// the next.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -56,38 +59,60 @@ __device__ __forceinline__ void tri_tile128(int idx, int T, int& ti, int& tj) {
   tj = ti + idx;
 }
 
+struct TileInfo {
+  int blk, isR, i0, j0, K;
+  bool skip;
+};
+
+// Tile t of the launch: stats tiles run over (block, L/R, upper-triangle
+// tile), apply tiles over (block, tile); tiles outside a ragged block's valid
+// range, or of a parameter flagged non-finite, are skipped by every role.
 template <int MODE>
-__global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap map_gk,
+__device__ __forceinline__ TileInfo decode_tile(int t, const TcArgs& a) {
+  const int T = (a.S + kTM - 1) / kTM;
+  TileInfo x{};
+  int ti, tj;
+  if (MODE == kStats) {
+    const int ntri = T * (T + 1) / 2;
+    x.blk = t / (2 * ntri);
+    const int r = t % (2 * ntri);
+    x.isR = r / ntri;
+    tri_tile128(r % ntri, T, ti, tj);
+  } else {
+    x.blk = t / (T * T);
+    const int r = t % (T * T);
+    ti = r / T;
+    tj = r % T;
+  }
+  const BlockDesc bd = a.blocks[x.blk];
+  x.i0 = ti * kTM;
+  x.j0 = tj * kTM;
+  if (MODE == kStats) {
+    const int side = x.isR ? bd.n : bd.m;
+    x.skip = x.i0 >= side || x.j0 >= side;
+    x.K = x.isR ? bd.m : bd.n;
+  } else {
+    x.skip = x.i0 >= bd.m || x.j0 >= bd.n;
+    x.K = (MODE == kApplyY) ? bd.n : bd.m;
+  }
+  x.skip = x.skip || a.flags[bd.param] != 0;
+  return x;
+}
+
+__host__ __device__ constexpr int ring_stages(int stage_bytes) {
+  return (192 * 1024) / stage_bytes < 2 ? 2 : ((192 * 1024) / stage_bytes > 8 ? 8 : (192 * 1024) / stage_bytes);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap map_gk,
                                                          const __grid_constant__ CUtensorMap map_gmn,
                                                          const __grid_constant__ CUtensorMap map_rk,
                                                          const __grid_constant__ CUtensorMap map_ymn,
-                                                         TcArgs args) {
+                                                         TcArgs args, int ntiles) {
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int blk = blockIdx.y;
-  const BlockDesc bd = args.blocks[blk];
-  if (args.flags[bd.param]) return;
   const int S = args.S;
-  const int T = (S + kTM - 1) / kTM;
 
-  // ---- what this CTA computes ----
-  int ti, tj, K, a_mn = 0, b_mn = 0, isR = 0;
-  if (MODE == kStats) {
-    isR = blockIdx.z;
-    tri_tile128(blockIdx.x, T, ti, tj);
-    const int side = isR ? bd.n : bd.m;
-    if (ti * kTM >= side || tj * kTM >= side) return;
-    K = isR ? bd.m : bd.n;
-    a_mn = b_mn = isR;
-  } else {
-    ti = blockIdx.x / T;
-    tj = blockIdx.x % T;
-    if (ti * kTM >= bd.m || tj * kTM >= bd.n) return;
-    K = (MODE == kApplyY) ? bd.n : bd.m;
-    b_mn = (MODE == kApplyP);
-  }
-  const int i0 = ti * kTM, j0 = tj * kTM;
-  const int nk = (K + kBKe - 1) / kBKe;
   // operand planes loaded and the (A plane, B plane) products kept, packed
   // two bits per product
   const bool g1 = args.planes_g == 1;
@@ -107,13 +132,15 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
     npass = 3; pas = (1u << 4); pbs = (1u << 2);          // h h, h l, l h
   }
   const int stage_bytes = (nA + nB) * kBoxBytes;
-  const int ST = stage_bytes <= 3 * kBoxBytes ? 3 : 2;
+  const int ST = ring_stages(stage_bytes);
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * stage_bytes);
   uint64_t* empty = full + ST;
-  uint64_t* accum = empty + ST;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* tfull = empty + ST;     // [2] accumulator ready for the epilogue
+  uint64_t* tempty = tfull + 2;     // [2] accumulator drained by the epilogue
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (tid == 0) {
@@ -121,12 +148,16 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    tc::mbar_init(accum, 1);
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull[a], 1);
+      tc::mbar_init(&tempty[a], 128);
+    }
+    tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 0) {
-    tc::tmem_alloc(tmem_slot, 128);
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 256);
     tc::tmem_relinquish();
   }
   __syncthreads();
@@ -135,161 +166,210 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
-    const CUtensorMap* mA = (MODE == kApplyP) ? &map_rk : (isR ? &map_gmn : &map_gk);
-    const CUtensorMap* mB = (MODE == kStats) ? (isR ? &map_gmn : &map_gk)
-                                             : (MODE == kApplyY ? &map_rk : &map_ymn);
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % ST;
-      if (kt >= ST && !tc::mbar_wait(&empty[s], ((kt / ST) - 1) & 1)) {
-        *abort_flag = 1;
-        atomicExch(args.err, tc::kErrTimeout);
-        break;
-      }
-      uint8_t* st = smem + s * stage_bytes;
-      tc::mbar_expect_tx(&full[s], stage_bytes);
-      const int k0 = kt * kBKe;
-      for (int pa = 0; pa < nA; ++pa) {
-        uint8_t* dst = st + pa * kBoxBytes;
-        if (MODE == kStats && isR) {          // A(i, k) = G[k][i]: two 64-wide boxes along i
-          tc::tma_load_3d(dst, mA, &full[s], i0, k0, pa * args.nblk + blk);
-          tc::tma_load_3d(dst + kBoxBytes / 2, mA, &full[s], i0 + 64, k0, pa * args.nblk + blk);
-        } else if (MODE == kApplyP) {         // A = L^{-1/p} planes
-          tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nmat + 2 * blk);
-        } else {                              // A = G rows
-          tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nblk + blk);
+    int g = 0;   // ring position, counted across tiles
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      const TileInfo x = decode_tile<MODE>(t, args);
+      if (x.skip) continue;
+      const int blk = x.blk, i0 = x.i0, j0 = x.j0, isR = x.isR;
+      const CUtensorMap* mA = (MODE == kApplyP) ? &map_rk : (isR ? &map_gmn : &map_gk);
+      const CUtensorMap* mB = (MODE == kStats) ? (isR ? &map_gmn : &map_gk)
+                                               : (MODE == kApplyY ? &map_rk : &map_ymn);
+      const int nk = (x.K + kBKe - 1) / kBKe;
+      for (int kt = 0; kt < nk; ++kt, ++g) {
+        const int s = g % ST;
+        if (g >= ST && !tc::mbar_wait(&empty[s], ((g / ST) - 1) & 1)) {
+          *abort_flag = 1;
+          atomicExch(args.err, tc::kErrTimeout);
+          break;
         }
-      }
-      for (int pb = 0; pb < nB; ++pb) {
-        uint8_t* dst = st + (nA + pb) * kBoxBytes;
-        if (MODE == kStats && isR) {
-          tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
-          tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
-        } else if (MODE == kStats) {
-          tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nblk + blk);
-        } else if (MODE == kApplyY) {         // B(k, j) = R^{-1/p}[j][k] (symmetric)
-          tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nmat + 2 * blk + 1);
-        } else {                              // B(k, j) = Y[k][j], MN-major
-          tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
-          tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
+        uint8_t* st = smem + s * stage_bytes;
+        tc::mbar_expect_tx(&full[s], stage_bytes);
+        const int k0 = kt * kBKe;
+        for (int pa = 0; pa < nA; ++pa) {
+          uint8_t* dst = st + pa * kBoxBytes;
+          if (MODE == kStats && isR) {          // A(i, k) = G[k][i]: two 64-wide boxes along i
+            tc::tma_load_3d(dst, mA, &full[s], i0, k0, pa * args.nblk + blk);
+            tc::tma_load_3d(dst + kBoxBytes / 2, mA, &full[s], i0 + 64, k0, pa * args.nblk + blk);
+          } else if (MODE == kApplyP) {         // A = L^{-1/p} planes
+            tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nmat + 2 * blk);
+          } else {                              // A = G rows
+            tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nblk + blk);
+          }
+        }
+        for (int pb = 0; pb < nB; ++pb) {
+          uint8_t* dst = st + (nA + pb) * kBoxBytes;
+          if (MODE == kStats && isR) {
+            tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
+            tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
+          } else if (MODE == kStats) {
+            tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nblk + blk);
+          } else if (MODE == kApplyY) {         // B(k, j) = R^{-1/p}[j][k] (symmetric)
+            tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nmat + 2 * blk + 1);
+          } else {                              // B(k, j) = Y[k][j], MN-major
+            tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
+            tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
+          }
         }
       }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
-    const uint32_t idesc = tc::idesc_bf16(kTM, kTM, a_mn, b_mn);
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % ST;
-      if (!tc::mbar_wait(&full[s], (kt / ST) & 1)) {
+    int g = 0, i = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      const TileInfo x = decode_tile<MODE>(t, args);
+      if (x.skip) continue;
+      const int a_mn = (MODE == kStats) ? x.isR : 0;
+      const int b_mn = (MODE == kStats) ? x.isR : (MODE == kApplyP);
+      const uint32_t idesc = tc::idesc_bf16(kTM, kTM, a_mn, b_mn);
+      const int acc = i & 1;
+      if (i >= 2 && !tc::mbar_wait(&tempty[acc], ((i >> 1) - 1) & 1)) {
         *abort_flag = 1;
         atomicExch(args.err, tc::kErrTimeout);
         break;
       }
       tc::fence_after_sync();
-      const uint32_t st = tc::smem_u32(smem + s * stage_bytes);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        for (int q = 0; q < npass; ++q) {
-          const int pa = (pas >> (2 * q)) & 3;
-          const int pb = (pbs >> (2 * q)) & 3;
-          const uint32_t sa = st + pa * kBoxBytes;
-          const uint32_t sb = st + (nA + pb) * kBoxBytes;
-          const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
-                                   : tc::smem_desc(sa + kk * 32, 16, 1024);
-          const uint64_t db = b_mn ? tc::smem_desc(sb + kk * 2048, 8192, 1024)
-                                   : tc::smem_desc(sb + kk * 32, 16, 1024);
-          tc::mma_bf16(tmem, da, db, idesc, (kt | kk | q) != 0);
+      const uint32_t dt = tmem + acc * kTM;
+      const int nk = (x.K + kBKe - 1) / kBKe;
+      bool ok = true;
+      for (int kt = 0; kt < nk; ++kt, ++g) {
+        const int s = g % ST;
+        if (!tc::mbar_wait(&full[s], (g / ST) & 1)) {
+          *abort_flag = 1;
+          atomicExch(args.err, tc::kErrTimeout);
+          ok = false;
+          break;
         }
+        tc::fence_after_sync();
+        const uint32_t st = tc::smem_u32(smem + s * stage_bytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          for (int q = 0; q < npass; ++q) {
+            const int pa = (pas >> (2 * q)) & 3;
+            const int pb = (pbs >> (2 * q)) & 3;
+            const uint32_t sa = st + pa * kBoxBytes;
+            const uint32_t sb = st + (nA + pb) * kBoxBytes;
+            const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
+                                     : tc::smem_desc(sa + kk * 32, 16, 1024);
+            const uint64_t db = b_mn ? tc::smem_desc(sb + kk * 2048, 8192, 1024)
+                                     : tc::smem_desc(sb + kk * 32, 16, 1024);
+            tc::mma_bf16(dt, da, db, idesc, (kt | kk | q) != 0);
+          }
+        }
+        tc::mma_commit(&empty[s]);
       }
-      tc::mma_commit(&empty[s]);
+      if (!ok) break;
+      tc::mma_commit(&tfull[acc]);
+      ++i;
     }
-    tc::mma_commit(accum);
-  }
-  __syncwarp();
-
-  // ---------------- epilogue: TMEM -> registers -> global ----------------
-  const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(accum, 0) && !*abort_flag);
-  tc::fence_after_sync();
-  const int r = i0 + warp * 32 + lane;         // output row owned by this thread
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-  if (ok) {
-    if (MODE == kStats) {
-      float* C = args.stats + (size_t)(2 * blk + isR) * S * S;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tc::tmem_ld32(trow + c * 32, v);
-        const int cb = j0 + c * 32;
-        if (r < S && cb < S) {
-          float4* row = reinterpret_cast<float4*>(C + (size_t)r * S + cb);
+    // every MMA this thread issued has landed before TMEM is released
+    tc::mma_commit(drain);
+    tc::mbar_wait(drain, 0);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> registers -> global ----------------
+    const int q = warp & 3;                      // TMEM lanes 32q .. 32q + 31
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const TileInfo x = decode_tile<MODE>(t, args);
+      if (x.skip) continue;
+      const int acc = i & 1;
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&tfull[acc], (i >> 1) & 1) && !*abort_flag);
+      if (!ok) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          atomicExch(args.err, tc::kErrTimeout);
+        }
+        break;
+      }
+      tc::fence_after_sync();
+      const int blk = x.blk, i0 = x.i0, j0 = x.j0;
+      const BlockDesc bd = args.blocks[blk];
+      const int r = i0 + q * 32 + lane;          // output row owned by this thread
+      const uint32_t trow = tmem + acc * kTM + ((uint32_t)(q * 32) << 16);
+      if (MODE == kStats) {
+        float* C = args.stats + (size_t)(2 * blk + x.isR) * S * S;
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(trow + c * 32, v);
+          const int cb = j0 + c * 32;
+          if (r < S && cb < S) {
+            float4* row = reinterpret_cast<float4*>(C + (size_t)r * S + cb);
+            float4 o[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 o = row[q];
-            o.x = fmaf(args.beta2, o.x, v[4 * q + 0]);
-            o.y = fmaf(args.beta2, o.y, v[4 * q + 1]);
-            o.z = fmaf(args.beta2, o.z, v[4 * q + 2]);
-            o.w = fmaf(args.beta2, o.w, v[4 * q + 3]);
-            row[q] = o;
+            for (int u = 0; u < 8; ++u) o[u] = row[u];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              o[u].x = fmaf(args.beta2, o[u].x, v[4 * u + 0]);
+              o[u].y = fmaf(args.beta2, o[u].y, v[4 * u + 1]);
+              o[u].z = fmaf(args.beta2, o[u].z, v[4 * u + 2]);
+              o[u].w = fmaf(args.beta2, o[u].w, v[4 * u + 3]);
+              row[u] = o[u];
+            }
           }
         }
-      }
-    } else if (MODE == kApplyY) {
-      uint16_t* yh = args.y + (size_t)blk * S * S;
-      uint16_t* yl = args.y + (size_t)(args.nblk + blk) * S * S;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tc::tmem_ld32(trow + c * 32, v);
-        const int cb = j0 + c * 32;
-        if (r < S && cb < S) {
-          uint32_t hw[16], lw[16];
+      } else if (MODE == kApplyY) {
+        uint16_t* yh = args.y + (size_t)blk * S * S;
+        uint16_t* yl = args.y + (size_t)(args.nblk + blk) * S * S;
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(trow + c * 32, v);
+          const int cb = j0 + c * 32;
+          if (r < S && cb < S) {
+            uint32_t hw[16], lw[16];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const uint16_t h0 = tc::bf16_bits_rn(v[2 * q]), h1 = tc::bf16_bits_rn(v[2 * q + 1]);
-            const uint16_t l0 = tc::bf16_bits_rn(v[2 * q] - tc::bf16_to_f(h0));
-            const uint16_t l1 = tc::bf16_bits_rn(v[2 * q + 1] - tc::bf16_to_f(h1));
-            hw[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-            lw[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-          }
-          uint4* dh = reinterpret_cast<uint4*>(yh + (size_t)r * S + cb);
-          uint4* dl = reinterpret_cast<uint4*>(yl + (size_t)r * S + cb);
+            for (int u = 0; u < 16; ++u) {
+              const uint16_t h0 = tc::bf16_bits_rn(v[2 * u]), h1 = tc::bf16_bits_rn(v[2 * u + 1]);
+              const uint16_t l0 = tc::bf16_bits_rn(v[2 * u] - tc::bf16_to_f(h0));
+              const uint16_t l1 = tc::bf16_bits_rn(v[2 * u + 1] - tc::bf16_to_f(h1));
+              hw[u] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+              lw[u] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+            }
+            uint4* dh = reinterpret_cast<uint4*>(yh + (size_t)r * S + cb);
+            uint4* dl = reinterpret_cast<uint4*>(yl + (size_t)r * S + cb);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            dh[q] = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
-            dl[q] = make_uint4(lw[4 * q], lw[4 * q + 1], lw[4 * q + 2], lw[4 * q + 3]);
+            for (int u = 0; u < 4; ++u) {
+              dh[u] = make_uint4(hw[4 * u], hw[4 * u + 1], hw[4 * u + 2], hw[4 * u + 3]);
+              dl[u] = make_uint4(lw[4 * u], lw[4 * u + 1], lw[4 * u + 2], lw[4 * u + 3]);
+            }
           }
         }
-      }
-    } else {
-      double ss = 0.0;
-      float* Pp = args.P + args.params[bd.param].offset;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tc::tmem_ld32(trow + c * 32, v);
-        const int cb = j0 + c * 32;
-        if (r < bd.m) {
-          float* dst = Pp + (bd.r0 + r) * bd.ld + bd.c0 + cb;
-          if (cb + 32 <= bd.n && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      } else {
+        double ss = 0.0;
+        float* Pp = args.P + args.params[bd.param].offset;
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(trow + c * 32, v);
+          const int cb = j0 + c * 32;
+          if (r < bd.m) {
+            float* dst = Pp + (bd.r0 + r) * bd.ld + bd.c0 + cb;
+            if (cb + 32 <= bd.n && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              for (int u = 0; u < 8; ++u)
+                reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ss += (double)v[e] * v[e];
-          } else {
+              for (int e = 0; e < 32; ++e) ss += (double)v[e] * v[e];
+            } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (cb + e < bd.n) {
-                dst[e] = v[e];
-                ss += (double)v[e] * v[e];
+              for (int e = 0; e < 32; ++e) {
+                if (cb + e < bd.n) {
+                  dst[e] = v[e];
+                  ss += (double)v[e] * v[e];
+                }
               }
             }
           }
         }
+        ss = warp_sum(ss);
+        if (lane == 0 && ss != 0.0) atomicAdd(&args.p2[bd.param], ss);
       }
-      ss = warp_sum(ss);
-      if (lane == 0 && ss != 0.0) atomicAdd(&args.p2[bd.param], ss);
+      tc::fence_before_sync();
+      tc::mbar_arrive(&tempty[acc]);
+      ++i;
     }
   }
+  __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 128);
+  if (warp == 1) tc::tmem_dealloc(tmem, 256);
 }
 
 // K1: gradients -> blocked, zero-padded bf16 planes.  grid: x = 2048-element
@@ -359,15 +439,24 @@ __global__ void split_kernel(const float* __restrict__ x, int64_t n, uint16_t* _
   }
 }
 
-int stage_count(int stage_bytes) { return stage_bytes <= 3 * kBoxBytes ? 3 : 2; }
-
 size_t smem_bytes(int nA, int nB) {
   const int sb = (nA + nB) * kBoxBytes;
-  return (size_t)stage_count(sb) * sb + 1024 + 256;
+  return (size_t)ring_stages(sb) * sb + 1024 + 256;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
 }
 
 template <int MODE>
-cudaError_t launch_mode(dim3 grid, size_t smem, const TcMaps& maps, const TcArgs& a, cudaStream_t s) {
+cudaError_t launch_mode(int ntiles, size_t smem, const TcMaps& maps, const TcArgs& a, cudaStream_t s) {
   static bool configured = false;   // per process; the attribute is per function
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -375,7 +464,8 @@ cudaError_t launch_mode(dim3 grid, size_t smem, const TcMaps& maps, const TcArgs
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  tc_gemm_kernel<MODE><<<grid, 128, smem, s>>>(maps.gk, maps.gmn, maps.rk, maps.ymn, a);
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  tc_gemm_kernel<MODE><<<grid, 192, smem, s>>>(maps.gk, maps.gmn, maps.rk, maps.ymn, a, ntiles);
   return cudaGetLastError();
 }
 
@@ -402,7 +492,7 @@ cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const i
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
   a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err;
   const int T = (S + kTM - 1) / kTM;
-  return launch_mode<kStats>(dim3(T * (T + 1) / 2, nblk, 2), smem_bytes(planes_g, planes_g), maps, a, s);
+  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, planes_g), maps, a, s);
 }
 
 cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
@@ -412,7 +502,7 @@ cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
   a.planes_g = planes_g; a.y = y; a.err = err;
   const int T = (S + kTM - 1) / kTM;
-  return launch_mode<kApplyY>(dim3(T * T, nblk), smem_bytes(planes_g == 1 ? 1 : 2, 2), maps, a, s);
+  return launch_mode<kApplyY>(nblk * T * T, smem_bytes(planes_g == 1 ? 1 : 2, 2), maps, a, s);
 }
 
 cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const ParamDesc* params,
@@ -423,7 +513,7 @@ cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const
   a.blocks = blocks; a.params = params; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
   a.planes_g = 2; a.P = P; a.p2 = p2; a.err = err;
   const int T = (S + kTM - 1) / kTM;
-  return launch_mode<kApplyP>(dim3(T * T, nblk), smem_bytes(2, 2), maps, a, s);
+  return launch_mode<kApplyP>(nblk * T * T, smem_bytes(2, 2), maps, a, s);
 }
 
 }  // namespace shampoo

@@ -90,6 +90,7 @@ size_t carve(unsigned char* base, int chunk, int S, NewtonWork* w, NewtonMat** m
   w->sched = c.take<double>((size_t)chunk * kSched);
   w->nsched = c.take<int>(chunk);
   w->resid = c.take<unsigned long long>(chunk);
+  w->fro2 = c.take<double>(chunk);
   w->prev = c.take<double>(chunk);
   w->worse = c.take<int>(chunk);
   w->active = nullptr;
