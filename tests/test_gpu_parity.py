@@ -273,3 +273,54 @@ def test_scaled_newton_takes_fewer_steps_than_plain():
         assert ok and 0 < iters[i] < k_plain, (i, iters[i], k_plain)
         ref = inverse_root(A32[i].astype(np.float64), 1e-6, 4)
         assert rel(X[i], ref) <= ROOT_TOL
+
+
+def run_subset(cfg, steps, interval, keep):
+    """Run the CUDA path on the whole parameter set of `cfg` and the oracle
+    on the parameters listed in `keep` only (parameters never interact: each
+    has its own statistics and its own graft scale).  Returns the worst
+    per-block relative errors of W and of the last step's dW."""
+    from shampoo_second_order_b200 import Shampoo
+    shapes = cfg["shapes"]
+    sub = [shapes[i] for i in keep]
+    o = ShampooOracle(sub, cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"], cfg["graft"],
+                      cfg["momentum"])
+    opt = Shampoo(shapes, cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"], cfg["graft"],
+                  cfg["momentum"], cfg["grad_dtype"])
+    W0 = wl.make_params(shapes, cfg["seed"])
+    Wd = [torch.from_numpy(w).cuda() for w in W0]
+    Wo = [W0[i].astype(np.float64) for i in keep]
+    for t in range(steps):
+        g = wl.make_grads(shapes, cfg["seed"], t, cfg["grad_std"], cfg["grad_dtype"])
+        roots = t % interval == 0
+        prev_d = [Wd[i].cpu().numpy().astype(np.float64) for i in keep]
+        prev_o = Wo
+        Wo = o.step(Wo, [g[i] for i in keep], cfg["lr"], roots)
+        opt.step(Wd, [to_dev(x, cfg["grad_dtype"]) for x in g], cfg["lr"], roots)
+        torch.cuda.synchronize()
+        del g
+    worst = {"dW": 0.0, "W": 0.0}
+    for k, i in enumerate(keep):
+        wd = Wd[i].cpu().numpy().astype(np.float64)
+        for sl in pieces(shapes[i], cfg["block_size"]):
+            worst["dW"] = max(worst["dW"], rel((wd - prev_d[k])[sl], (Wo[k] - prev_o[k])[sl]))
+            worst["W"] = max(worst["W"], rel(wd[sl], Wo[k][sl]))
+    opt.close()
+    return worst
+
+
+def test_transformer_big_full_set_sampled_parameters():
+    """The ~285M-parameter Transformer-big set (b = 1024, fp32 gradients,
+    momentum 0.9) runs whole on the GPU; layer 0's query, FFN-in and FFN-out
+    weights are checked against the oracle over 3 steps (roots at 1 and 3)."""
+    c = wl.CONFIGS["transformer_big_b1024"]
+    w = run_subset(c, steps=3, interval=2, keep=[0, 4, 5])
+    assert w["dW"] <= STEP_TOL and w["W"] <= STEP_TOL, w
+
+
+def test_resnet50_full_set():
+    """Every ResNet-50 weight (1576 blocks of <= 128, 430 vector segments,
+    fp32 gradients) against the oracle over 3 steps (roots at 1 and 3)."""
+    c = wl.CONFIGS["resnet50_b128"]
+    w = run_subset(c, steps=3, interval=2, keep=list(range(len(c["shapes"]))))
+    assert w["dW"] <= STEP_TOL and w["W"] <= STEP_TOL, w
