@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(256) update_kernel(
     float4* w4 = reinterpret_cast<float4*>(w);
     const float4* p4 = reinterpret_cast<const float4*>(pp);
     float4* m4 = reinterpret_cast<float4*>(mm);
+#pragma unroll 4
     for (int v = threadIdx.x; v < n4; v += blockDim.x) {
       const float4 p = p4[v];
       float4 x = w4[v];

@@ -101,6 +101,8 @@ __device__ __forceinline__ void dmma_tile(const double* __restrict__ A, const do
     cp_async_commit();
   };
   const int nk = S / kBK;
+  // on a diagonal tile the lower-left 32 x 32 block mirrors the upper-right one
+  const bool idle = (i0 == j0) && wm == 1 && wn == 0;
   load(0, 0);
   for (int kt = 0; kt < nk; ++kt) {
     if (kt + 1 < nk) {
@@ -112,7 +114,7 @@ __device__ __forceinline__ void dmma_tile(const double* __restrict__ A, const do
     __syncthreads();
     const int st = kt & 1;
 #pragma unroll
-    for (int kk = 0; kk < kBK; kk += 4) {
+    for (int kk = 0; kk < kBK && !idle; kk += 4) {
       double a[4], b[4];
 #pragma unroll
       for (int mi = 0; mi < 4; ++mi) a[mi] = sm.As[st][wm * 32 + mi * 8 + g][kk + t];
@@ -127,12 +129,24 @@ __device__ __forceinline__ void dmma_tile(const double* __restrict__ A, const do
   }
 }
 
-// Store the tile to C at (i0, j0) and, off the diagonal, its transpose at (j0, i0).
+// How a warp's 32 x 32 block of a tile is stored: on a diagonal tile the
+// lower-left warp computes nothing (its block mirrors the upper-right one);
+// every block off the matrix diagonal is also written transposed.
+__device__ __forceinline__ int warp_weight(int i0, int j0) {
+  const int warp = threadIdx.x >> 5, wm = warp >> 1, wn = warp & 1;
+  if (i0 != j0) return 2;            // off-diagonal tile: block and mirror
+  if (wm == 1 && wn == 0) return 0;  // idle
+  return (wm == 0 && wn == 1) ? 2 : 1;
+}
+
+// Store the tile to C at (i0, j0) and its mirror image where it has one.
 __device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0, int j0,
                                           const double acc[4][4][2]) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int wm = warp >> 1, wn = warp & 1;
+  const int wgt = warp_weight(i0, j0);
+  if (wgt == 0) return;
 #pragma unroll
   for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
@@ -140,7 +154,7 @@ __device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0,
       const int r = i0 + wm * 32 + mi * 8 + g;
       const int c = j0 + wn * 32 + ni * 8 + 2 * t;
       *reinterpret_cast<double2*>(C + (size_t)r * S + c) = make_double2(acc[mi][ni][0], acc[mi][ni][1]);
-      if (i0 != j0) {
+      if (wgt == 2) {
         C[(size_t)c * S + r] = acc[mi][ni][0];
         C[(size_t)(c + 1) * S + r] = acc[mi][ni][1];
       }
@@ -490,6 +504,7 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
   const int wm = warp >> 1, wn = warp & 1;
   const int n = mats[m].size;
   const double pinv = 1.0 / p;
+  const double wgt = warp_weight(i0, j0);   // 0: idle block, 2: block and mirror
   double dev = 0.0, f2 = 0.0;
 #pragma unroll
   for (int mi = 0; mi < 4; ++mi)
@@ -500,11 +515,10 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
         const int r = i0 + wm * 32 + mi * 8 + g;
         const int c = j0 + wn * 32 + ni * 8 + 2 * t + e;
         const double d = (r == c) ? 1.0 : 0.0;
-        double x = (r < n && c < n) ? fabs(acc[mi][ni][e] - d) : 0.0;
+        double x = (wgt > 0 && r < n && c < n) ? fabs(acc[mi][ni][e] - d) : 0.0;
         if (!(x <= DBL_MAX)) x = INFINITY;
         dev = fmax(dev, x);
-        // off-diagonal tiles stand for their mirror image too
-        f2 += (i0 == j0 ? 1.0 : 2.0) * x * x;
+        f2 += wgt * x * x;                       // mirrored blocks count twice
         acc[mi][ni][e] = ((p + 1) * d - sn * acc[mi][ni][e]) * pinv;
       }
   store_sym(w.T + base, S, i0, j0, acc);
@@ -617,7 +631,8 @@ void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, co
 }
 
 void launch_newton_lanczos(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {
-  newton_lanczos_kernel<<<nm, 512, 0, s>>>(mats, S, w);
+  const int threads = S <= 128 ? 128 : (S <= 256 ? 256 : 512);   // one warp per row at a time
+  newton_lanczos_kernel<<<nm, threads, 0, s>>>(mats, S, w);
 }
 
 void launch_newton_t0(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(256) diag_update_kernel(
   const bool al = aligned16(g, c.start, bf16);
   double s = 0.0;
   const int n4 = c.len >> 2;
+#pragma unroll 4
   for (int v = threadIdx.x; v < n4; v += blockDim.x) {
     const float4 x = grad4(g, c.start + 4 * (int64_t)v, bf16, al);
     float4 o = reinterpret_cast<float4*>(ap)[v];

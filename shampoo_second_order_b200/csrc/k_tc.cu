@@ -388,25 +388,67 @@ __global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict
   const int64_t base = (bd.r0 + i) * bd.ld + bd.c0;
   int bad = 0;
   if (i < bd.m) {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int jj = j + q;
-      if (jj < bd.n) {
-        uint16_t h, m = 0, l = 0;
-        if (bf16) {
-          h = __ldg(reinterpret_cast<const uint16_t*>(g) + base + jj);
-          bad |= (h & 0x7F80) == 0x7F80;
+    if (j + 8 <= bd.n) {   // a whole run of 8: vector loads when aligned
+      float x[8];
+      if (bf16) {
+        const uint16_t* src = reinterpret_cast<const uint16_t*>(g) + base + j;
+        uint32_t u[4];
+        if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
+          u[0] = v.x; u[1] = v.y; u[2] = v.z; u[3] = v.w;
         } else {
-          const float x = __ldg(reinterpret_cast<const float*>(g) + base + jj);
-          bad |= !isfinite(x);
-          h = tc::bf16_bits_rn(x);
-          const float r1 = x - tc::bf16_to_f(h);        // exact
-          m = tc::bf16_bits_rn(r1);
-          l = tc::bf16_bits_rn(r1 - tc::bf16_to_f(m));  // exact remainder, rounded
+          for (int q = 0; q < 4; ++q)
+            u[q] = (uint32_t)__ldg(src + 2 * q) | ((uint32_t)__ldg(src + 2 * q + 1) << 16);
         }
-        hw[q >> 1] |= (uint32_t)h << (16 * (q & 1));
-        mw[q >> 1] |= (uint32_t)m << (16 * (q & 1));
-        lw[q >> 1] |= (uint32_t)l << (16 * (q & 1));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          hw[q] = u[q];
+          bad |= ((u[q] & 0x7F80u) == 0x7F80u) | ((u[q] & 0x7F800000u) == 0x7F800000u);
+        }
+      } else {
+        const float* src = reinterpret_cast<const float*>(g) + base + j;
+        if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+          const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+          const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+          x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) x[q] = __ldg(src + q);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          bad |= !isfinite(x[q]);
+          const uint16_t h = tc::bf16_bits_rn(x[q]);
+          const float r1 = x[q] - tc::bf16_to_f(h);        // exact
+          const uint16_t m = tc::bf16_bits_rn(r1);
+          const uint16_t l = tc::bf16_bits_rn(r1 - tc::bf16_to_f(m));
+          hw[q >> 1] |= (uint32_t)h << (16 * (q & 1));
+          mw[q >> 1] |= (uint32_t)m << (16 * (q & 1));
+          lw[q >> 1] |= (uint32_t)l << (16 * (q & 1));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int jj = j + q;
+        if (jj < bd.n) {
+          uint16_t h, m = 0, l = 0;
+          if (bf16) {
+            h = __ldg(reinterpret_cast<const uint16_t*>(g) + base + jj);
+            bad |= (h & 0x7F80) == 0x7F80;
+          } else {
+            const float x = __ldg(reinterpret_cast<const float*>(g) + base + jj);
+            bad |= !isfinite(x);
+            h = tc::bf16_bits_rn(x);
+            const float r1 = x - tc::bf16_to_f(h);        // exact
+            m = tc::bf16_bits_rn(r1);
+            l = tc::bf16_bits_rn(r1 - tc::bf16_to_f(m));  // exact remainder, rounded
+          }
+          hw[q >> 1] |= (uint32_t)h << (16 * (q & 1));
+          mw[q >> 1] |= (uint32_t)m << (16 * (q & 1));
+          lw[q >> 1] |= (uint32_t)l << (16 * (q & 1));
+        }
       }
     }
   }
