@@ -126,45 +126,59 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons of one GPU, polled through NVML every
+    2 ms on a background thread while the timed region runs (nvidia-smi's
+    fastest loop is too slow for a region of tens of milliseconds)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
-    def __init__(self, uuid=None):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
-        if uuid:
-            cmd += ["-i", uuid]
+    def __init__(self, uuid=None, index=0):
+        import threading
+        self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
+        self.stop_flag = threading.Event()
         try:
-            self.p = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.p = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            h = None
+            if uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+                except Exception:
+                    h = None
+            self.h = h or pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # no NVML: report why
+            self.nv, self.err = None, str(e)
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = get(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.002)
 
     def stop(self):
-        if self.p is None:
-            return None
-        self.p.terminate()
-        try:
-            self.p.wait(5)
-        except subprocess.TimeoutExpired:
-            self.p.kill()
-        self.f.flush()
-        rows = []
-        with open(self.f.name) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.f.name)
-        if not rows:
-            return {"error": "no nvidia-smi samples"}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if self.nv is None:
+            return {"error": self.err}
+        self.stop_flag.set()
+        self.t.join(timeout=2)
+        if not self.samples:
+            return {"error": self.err or "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "NVML, 2 ms"}
 
 
 def gpu_uuid(torch, dev):
@@ -193,6 +207,32 @@ def fp64_peak_tflops(torch, dev):
     return 2 * n ** 3 / (best * 1e-3) / 1e12
 
 
+def tc_work(cfg, kernel):
+    """Algorithmic (flops, bytes) of one launch of a tensor-core kernel over
+    the whole parameter set: flops as bf16 MMA work (products kept x the
+    exact flop count), bytes as the minimum HBM traffic (each operand read once,
+    each output written once; statistics read and written on their
+    upper-triangle 128-tiles)."""
+    b = cfg["block_size"]
+    blks, _ = blocks_of(cfg)
+    f32 = cfg["grad_dtype"] == "f32"
+    planes = 3 if f32 else 1
+    T = (b + 127) // 128
+    tri = T * (T + 1) // 2 * 128 * 128 * 4          # bytes of one statistic's upper tiles
+    if kernel == "stats_tc":
+        passes = 6 if f32 else 1
+        fl = sum(m * (m + 1) * n + n * (n + 1) * m for m, n in blks) * passes
+        by = sum(2 * planes * m * n for m, n in blks) + len(blks) * 2 * 2 * tri
+    elif kernel == "apply_y_tc":
+        passes = 3 if f32 else 2
+        fl = sum(2 * m * n * n for m, n in blks) * passes
+        by = sum(2 * min(planes, 2) * m * n + 2 * 2 * n * n + 2 * 2 * m * n for m, n in blks)
+    else:   # apply_p_tc
+        fl = sum(2 * m * m * n for m, n in blks) * 3
+        by = sum(2 * 2 * m * m + 2 * 2 * m * n + 4 * m * n for m, n in blks)
+    return fl, by
+
+
 def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak):
     """Achieved vs peak for the kernel with the largest share of device time."""
     names = {k: v for k, v in prof.items() if v[1] > 0}
@@ -200,7 +240,9 @@ def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak):
         return None, None
     top = max(names, key=lambda k: names[k][1])
     launches, ms = names[top]
+    sec = ms * 1e-3
     hbm = peaks["hbm_gbs"]
+    bf16 = peaks["bf16_tflops"]
     blks, segs = blocks_of(cfg)
     el = numel(cfg)
     gbytes = 2 if cfg["grad_dtype"] == "bf16" else 4
@@ -208,31 +250,36 @@ def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak):
     if top.startswith("newton_step"):
         a, b, c = newton_flops(cfg, iters_sum, per_kernel=True)
         fl = {"newton_step_a": a, "newton_step_b": b, "newton_step_c": c}[top]
-        work = ("tensor", fl / 1e12 / (ms * 1e-3), fp64_peak, "TFLOP/s", fl / max(launches, 1))
-    elif top == "stats_blocks":
-        fl = (stats_flops(cfg) - sum(l * (l + 1) for l in segs)) * steps
-        work = ("alu", fl / 1e12 / (ms * 1e-3), 74.4, "TFLOP/s", fl / max(launches, 1))
-    elif top in ("precond_y", "precond_p"):
-        fl = sum(2 * m * n * (n if top == "precond_y" else m) for m, n in blks) * steps
-        work = ("alu", fl / 1e12 / (ms * 1e-3), 74.4, "TFLOP/s", fl / max(launches, 1))
+        work = ("tensor", fl / 1e12 / sec, fp64_peak, "TFLOP/s", fl / max(launches, 1),
+                "cuBLAS DGEMM (fp64) measured in this run")
+    elif top in ("stats_tc", "apply_y_tc", "apply_p_tc"):
+        fl, by = tc_work(cfg, top)
+        fl, by = fl * launches, by * launches
+        ft, fh = fl / 1e12 / sec / bf16, by / 1e9 / sec / hbm
+        if ft >= fh:
+            work = ("tensor", fl / 1e12 / sec, bf16, "TFLOP/s", fl / launches,
+                    "MEASURED_PEAKS.json bf16_tflops (burst)")
+        else:
+            work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / launches, "MEASURED_PEAKS.json hbm_gbs")
+    elif top == "newton_lanczos":
+        by = sum(12 * 8 * n * n for n, _ in matrix_sizes(cfg)) * n_root_steps
+        work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")
     elif top == "update":
         by = el * (4 + 8 + (8 if cfg["momentum"] else 0)) * steps
-        work = ("hbm", by / 1e9 / (ms * 1e-3), hbm, "GB/s", by / max(launches, 1))
-    elif top in ("dnorm", "diag_update", "check_finite"):
-        per = {"dnorm": gbytes + 4, "diag_update": gbytes + 8, "check_finite": gbytes}[top]
+        work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")
+    elif top in ("dnorm", "diag_update", "check_finite", "gather"):
+        per = {"dnorm": gbytes + 4, "diag_update": gbytes + 8, "check_finite": gbytes,
+               "gather": gbytes + (6 if gbytes == 4 else 2)}[top]
         by = el * per * steps
-        work = ("hbm", by / 1e9 / (ms * 1e-3), hbm, "GB/s", by / max(launches, 1))
+        work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")
     if work is None:
         return top, None
-    bound, ach, peak, unit, per_launch = work
+    bound, ach, peak, unit, per_launch, src = work
     tr = TRAFFIC_PER_LAUNCH.get(top)
     return top, {"kernel": top, "bound": bound, "achieved": round(ach, 3), "peak": round(peak, 2),
                  "unit": unit, "frac": round(ach / peak, 4), "traffic": tr,
                  "algorithmic_per_launch": per_launch, "launches": launches,
-                 "avg_launch_ms": round(ms / launches, 5),
-                 "peak_source": "cuBLAS DGEMM measured in this run" if bound == "tensor" else
-                 ("MEASURED_PEAKS.json hbm_gbs" if bound == "hbm" else
-                  "fp32 FMA units: 148 SMs x 128 lanes x 2 flop x 1.965 GHz")}
+                 "avg_launch_ms": round(ms / launches, 5), "peak_source": src}
 
 
 # ---------------------------------------------------------------------------
@@ -257,6 +304,26 @@ def oracle_sample(cfg, n_steps):
         W = o.apply(W, g, cfg["lr"])
     t_sa = (time.perf_counter() - t0) / n_steps
     return t_sa + t_root / cfg["root_interval"], t_root, t_sa
+
+
+def pages_design_root_ms(cfg, n_sample=4):
+    """The pages' root route on host cores: fp64 coupled Newton (the
+    oracle's CPU copy) on the first n_sample statistics after 2 steps,
+    extrapolated to every statistic of the set by n^3."""
+    from oracle import ShampooOracle, coupled_newton_inverse_root
+    o = ShampooOracle(cfg["shapes"], cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"],
+                      cfg["graft"], cfg["momentum"])
+    for t in range(2):
+        o.update_stats(wl.make_grads(cfg["shapes"], cfg["seed"], t, cfg["grad_std"], cfg["grad_dtype"]))
+    mats = o.matrices()
+    t0 = time.perf_counter()
+    done = 0.0
+    for A, p in mats[:n_sample]:
+        coupled_newton_inverse_root(A, cfg["eps"], p)
+        done += A.shape[0] ** 3
+    el = time.perf_counter() - t0
+    total = sum(A.shape[0] ** 3 for A, _ in mats)
+    return el * total / done * 1e3
 
 
 def blas_threads():
@@ -391,7 +458,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         t_step, t_root, t_sa = oracle_sample(cfg, 2)
-        cpu = {"t_step_s": t_step, "t_root_s": t_root, "t_stats_apply_s": t_sa}
+        cpu = {"t_step_s": t_step, "t_root_s": t_root, "t_stats_apply_s": t_sa,
+               "pages_root_ms": pages_design_root_ms(cfg)}
 
     import torch
     import torch.distributed as dist
@@ -441,7 +509,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     uuid = gpu_uuid(torch, dev)
-    clocks = ClockSampler(uuid)
+    clocks = ClockSampler(uuid, local)
     opt.profile_enable(True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
@@ -544,7 +612,11 @@ def main():
                         "kind": "oracle",
                         "sample": ("fp64 numpy oracle on the full workload: 2 steps of stats+apply and 1 "
                                    "root step (eigh), amortised over the root interval"),
-                        "ms_per_step": cpu["t_step_s"] * 1e3}
+                        "ms_per_step": cpu["t_step_s"] * 1e3,
+                        "root_step_ms_eigh": cpu["t_root_s"] * 1e3,
+                        "root_step_ms_pages_design": round(cpu["pages_root_ms"], 1),
+                        "pages_design": ("fp64 coupled Newton on host cores for every statistic "
+                                         "(timed on 4, extrapolated by n^3)")}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
