@@ -332,17 +332,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor [depth][S][S] with a box of box_x (inner) x box_y rows.
-bool encode_planes(CUtensorMap* m, void* base, int S, int64_t depth, int box_x, int box_y) {
+// 3-D tensor [depth][S][S] of bf16 (or fp32) with a box of box_x (inner) x
+// box_y rows, 128-byte swizzle.
+bool encode_planes(CUtensorMap* m, void* base, int S, int64_t depth, int box_x, int box_y,
+                   bool fp32 = false) {
   auto fn = encode_fn();
   if (!fn || depth < 1) return false;
+  const cuuint64_t esz = fp32 ? 4 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)S, (cuuint64_t)S, (cuuint64_t)depth};
-  cuuint64_t strides[2] = {(cuuint64_t)S * 2, (cuuint64_t)S * S * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)S * esz, (cuuint64_t)S * S * esz};
   cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
+            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // A kernel that gave up on a wait leaves a code in the error word.
@@ -546,7 +549,8 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
       !(encode_planes(&ctx->maps.gk, ctx->gblk, b, ctx->planes_g * nblk64, 64, 128) &&
         encode_planes(&ctx->maps.gmn, ctx->gblk, b, ctx->planes_g * nblk64, 64, 64) &&
         encode_planes(&ctx->maps.rk, ctx->rplanes, b, 2 * (int64_t)ctx->nmat, 64, 128) &&
-        encode_planes(&ctx->maps.ymn, ctx->yplanes, b, 2 * nblk64, 64, 64))) {
+        encode_planes(&ctx->maps.ymn, ctx->yplanes, b, 2 * nblk64, 64, 64) &&
+        encode_planes(&ctx->maps.ck, ctx->stats, b, ctx->nmat, 32, 128, true))) {
     shampoo_destroy(ctx);
     return fail(nullptr, SHAMPOO_ECUDA, "cuTensorMapEncodeTiled failed");
   }

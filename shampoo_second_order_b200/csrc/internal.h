@@ -51,8 +51,9 @@ struct NewtonMat {
 //  gmn  the same tensor, box 64 x 64 (MN-major loads of G^T)
 //  rk   root planes [2*nmat][S][S] (hi then lo), box 64 x 128
 //  ymn  Y = G R^{-1/p} planes [2*nblk][S][S], box 64 x 64 (MN-major)
+//  ck   statistics fp32 [nmat][S][S], box 32 x 128 (the update's read-modify-write)
 struct TcMaps {
-  CUtensorMap gk, gmn, rk, ymn;
+  CUtensorMap gk, gmn, rk, ymn, ck;
 };
 
 // ---------------- tensor-core kernels (k_tc.cu) ----------------

@@ -99,8 +99,13 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const TcArgs& a) {
   return x;
 }
 
-__host__ __device__ constexpr int ring_stages(int stage_bytes) {
-  return (192 * 1024) / stage_bytes < 2 ? 2 : ((192 * 1024) / stage_bytes > 8 ? 8 : (192 * 1024) / stage_bytes);
+constexpr int kCTileBytes = 128 * 128 * 4;   // one fp32 statistics tile (4 boxes of 32 columns)
+
+// Ring stages that fit beside the 64 KB statistics tile when the update
+// stages it in shared memory (cstage), else beside nothing.
+__host__ __device__ constexpr int ring_stages(int stage_bytes, bool cstage = false) {
+  const int budget = (cstage ? 224 * 1024 : 192 * 1024) - (cstage ? kCTileBytes : 0);
+  return budget / stage_bytes < 2 ? 2 : (budget / stage_bytes > 8 ? 8 : budget / stage_bytes);
 }
 
 template <int MODE>
@@ -108,6 +113,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
                                                          const __grid_constant__ CUtensorMap map_gmn,
                                                          const __grid_constant__ CUtensorMap map_rk,
                                                          const __grid_constant__ CUtensorMap map_ymn,
+                                                         const __grid_constant__ CUtensorMap map_ck,
                                                          TcArgs args, int ntiles) {
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -132,15 +138,21 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     npass = 3; pas = (1u << 4); pbs = (1u << 2);          // h h, h l, l h
   }
   const int stage_bytes = (nA + nB) * kBoxBytes;
-  const int ST = ring_stages(stage_bytes);
+  // bf16 statistics: the old statistics tile comes in by TMA during the main
+  // loop, is updated in shared memory and goes back out by TMA
+  const bool cstage = (MODE == kStats) && g1;
+  const int ST = ring_stages(stage_bytes, cstage);
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * stage_bytes);
+  uint8_t* cbuf = smem + ST * stage_bytes;     // the 64 KB statistics tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + (cstage ? kCTileBytes : 0));
   uint64_t* empty = full + ST;
   uint64_t* tfull = empty + ST;     // [2] accumulator ready for the epilogue
   uint64_t* tempty = tfull + 2;     // [2] accumulator drained by the epilogue
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* cfull = drain + 1;      // statistics tile loaded
+  uint64_t* cready = cfull + 1;     // all epilogue threads wrote the tile (count 128)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (tid == 0) {
@@ -153,6 +165,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       tc::mbar_init(&tempty[a], 128);
     }
     tc::mbar_init(drain, 1);
+    tc::mbar_init(cfull, 1);
+    tc::mbar_init(cready, 128);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -268,6 +282,24 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     // ---------------- epilogue: TMEM -> registers -> global ----------------
     const int q = warp & 3;                      // TMEM lanes 32q .. 32q + 31
     int i = 0;
+    int c_loads = 0;   // statistics-tile loads issued (phase of the next one)
+    // bf16 statistics: lane 0 of warp 2 owns the shared statistics tile; it
+    // loads the first tile's old statistics now and each next tile's right
+    // after storing the previous one, while that tile's main loop runs
+    auto load_c = [&](int from) {
+      for (int t = from; t < ntiles; t += gridDim.x) {
+        const TileInfo y = decode_tile<MODE>(t, args);
+        if (y.skip) continue;
+        const int nbox = (S - y.j0 + 31) / 32 < 4 ? (S - y.j0 + 31) / 32 : 4;
+        tc::mbar_expect_tx(cfull, nbox * (kCTileBytes / 4));
+        for (int c = 0; c < nbox; ++c)
+          tc::tma_load_3d(cbuf + c * (kCTileBytes / 4), &map_ck, cfull, y.j0 + 32 * c, y.i0,
+                          2 * y.blk + y.isR);
+        ++c_loads;
+        return;
+      }
+    };
+    if (cstage && warp == 2 && lane == 0) load_c(blockIdx.x);
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       const TileInfo x = decode_tile<MODE>(t, args);
       if (x.skip) continue;
@@ -285,7 +317,48 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       const BlockDesc bd = args.blocks[blk];
       const int r = i0 + q * 32 + lane;          // output row owned by this thread
       const uint32_t trow = tmem + acc * kTM + ((uint32_t)(q * 32) << 16);
-      if (MODE == kStats) {
+      if (MODE == kStats && cstage) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(cfull, i & 1))) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            atomicExch(args.err, tc::kErrTimeout);
+          }
+          break;
+        }
+        const int rl = q * 32 + lane;            // tile-local row
+        const int nbox = (S - j0 + 31) / 32 < 4 ? (S - j0 + 31) / 32 : 4;
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(trow + c * 32, v);
+          if (c >= nbox) continue;
+          // row rl of box c: 8 chunks of 16 B, chunk j stored at j ^ (rl & 7)
+          uint8_t* row = cbuf + c * (kCTileBytes / 4) + rl * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4* p4 = reinterpret_cast<float4*>(row + ((j ^ (rl & 7)) << 4));
+            float4 o = *p4;
+            o.x = fmaf(args.beta2, o.x, v[4 * j + 0]);
+            o.y = fmaf(args.beta2, o.y, v[4 * j + 1]);
+            o.z = fmaf(args.beta2, o.z, v[4 * j + 2]);
+            o.w = fmaf(args.beta2, o.w, v[4 * j + 3]);
+            *p4 = o;
+          }
+        }
+        tc::fence_proxy_async_smem();            // my writes, before the TMA store reads them
+        tc::mbar_arrive(cready);
+        if (warp == 2 && lane == 0) {
+          if (!tc::mbar_wait(cready, i & 1)) {
+            *abort_flag = 1;
+            atomicExch(args.err, tc::kErrTimeout);
+          } else {
+            for (int c = 0; c < nbox; ++c)
+              tc::tma_store_3d(&map_ck, cbuf + c * (kCTileBytes / 4), j0 + 32 * c, i0, 2 * blk + x.isR);
+            tc::bulk_commit();
+            tc::bulk_wait_read0();                 // the tile buffer is free again
+            load_c(t + gridDim.x);
+          }
+        }
+      } else if (MODE == kStats) {
         float* C = args.stats + (size_t)(2 * blk + x.isR) * S * S;
         for (int c = 0; c < 4; ++c) {
           float v[32];
@@ -365,7 +438,10 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       tc::mbar_arrive(&tempty[acc]);
       ++i;
     }
+    // after an abort a statistics-tile load may still be in flight: let it land
+    if (cstage && warp == 2 && lane == 0 && c_loads > i) tc::mbar_wait(cfull, (c_loads - 1) & 1);
   }
+  if (cstage && warp == 2 && lane == 0) tc::bulk_wait0();   // statistics stores complete
   __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
@@ -481,9 +557,9 @@ __global__ void split_kernel(const float* __restrict__ x, int64_t n, uint16_t* _
   }
 }
 
-size_t smem_bytes(int nA, int nB) {
+size_t smem_bytes(int nA, int nB, bool cstage = false) {
   const int sb = (nA + nB) * kBoxBytes;
-  return (size_t)ring_stages(sb) * sb + 1024 + 256;
+  return (size_t)ring_stages(sb, cstage) * sb + (cstage ? kCTileBytes : 0) + 1024 + 256;
 }
 
 int sm_count() {
@@ -502,12 +578,12 @@ cudaError_t launch_mode(int ntiles, size_t smem, const TcMaps& maps, const TcArg
   static bool configured = false;   // per process; the attribute is per function
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         200 * 1024);
+                                         227 * 1024);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   const int grid = ntiles < sm_count() ? ntiles : sm_count();
-  tc_gemm_kernel<MODE><<<grid, 192, smem, s>>>(maps.gk, maps.gmn, maps.rk, maps.ymn, a, ntiles);
+  tc_gemm_kernel<MODE><<<grid, 192, smem, s>>>(maps.gk, maps.gmn, maps.rk, maps.ymn, maps.ck, a, ntiles);
   return cudaGetLastError();
 }
 
@@ -534,7 +610,8 @@ cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const i
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
   a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err;
   const int T = (S + kTM - 1) / kTM;
-  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, planes_g), maps, a, s);
+  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, planes_g, planes_g == 1),
+                             maps, a, s);
 }
 
 cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
