@@ -441,6 +441,7 @@ def main():
                     help="batched_roots_512 only: number of matrices (default 256)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-async", action="store_true")
     args = ap.parse_args()
     if args.config == "batched_roots_512":
         return roots_bench(args)
@@ -471,7 +472,9 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300))
 
-    stream = torch.cuda.Stream(device=dev)
+    # the steps' stream outranks the library's root stream (lowest priority),
+    # so asynchronous root work yields to the steps
+    stream = torch.cuda.Stream(device=dev, priority=-1)
     peaks, peak_src = measured_peaks()
     with torch.cuda.stream(stream):
         fp64_peak = fp64_peak_tflops(torch, dev)
@@ -599,6 +602,47 @@ def main():
                "ms_per_step": e2e_ms / args.steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "copies": "pinned host; uploads and downloads on two copy streams, overlapped with compute"}
 
+    # ---- asynchronous roots: the same K steps with the root job queued on the
+    # library's low-priority stream after step 0's statistics and swapped in by
+    # a later apply; the region ends when the job has been installed ----
+    async_line = None
+    if not args.no_async:
+        K = args.steps
+        sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        gen0 = opt.roots_generation()
+        installed_at = None
+        n_jobs = 0
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            for j in range(K):
+                flush.zero_()
+                sev[j][0].record(stream)
+                opt.update_stats(G[j % NG])
+                if j % interval == 0:
+                    n_jobs += int(opt.compute_roots_async())
+                opt.apply(W, G[j % NG], lr)
+                sev[j][1].record(stream)
+                if installed_at is None and opt.roots_generation() > gen0:
+                    installed_at = j
+            if opt.install_roots(wait=True) and installed_at is None:
+                installed_at = K
+            a1.record(stream)
+        stream.synchronize()
+        async_ms = max_over_ranks(a0.elapsed_time(a1), dist if world > 1 else None, dev)
+        its = opt.root_iterations()
+        fl = K * (stats_flops(cfg) + apply_flops(cfg)) + n_jobs * newton_flops(
+            cfg, [b if b >= 0 else -1 - b for b in its])
+        st_ms = sorted(s_.elapsed_time(e_) for s_, e_ in sev)
+        async_line = {"value": job_tflops(fl, world, async_ms), "unit": UNIT, "ms_per_step": async_ms / K,
+                      "root_jobs": n_jobs, "installed_at_step": installed_at,
+                      "step_ms_median": st_ms[len(st_ms) // 2], "step_ms_max": st_ms[-1],
+                      "sync_step_ms_max": max(s_.elapsed_time(e_) for s_, e_ in ev),
+                      "streams": "steps at high priority; roots on the library's lowest-priority stream"}
+
     top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak)
 
     if rank == 0:
@@ -625,7 +669,8 @@ def main():
                        "grad_dtype": cfg["grad_dtype"], "root_interval": interval,
                        "root_steps_timed": n_root, "l2": "flushed between steps (256 MiB write)",
                        "parallelism": f"replicas x{world}"},
-            "roofline": roof, "cpu_baseline": cpu_line, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roof, "cpu_baseline": cpu_line, "e2e": e2e, "async_roots": async_line,
+            "gpu_launches": launches,
             "clocks": clk, "kernels": phase, "fp64_gemm_peak_tflops": round(fp64_peak, 2),
             "peaks_source": peak_src,
             "flops_per_step": {"stats": stats_flops(cfg), "apply": apply_flops(cfg),

@@ -49,7 +49,8 @@ typedef enum {
   SHAMPOO_ECUDA = 3,          /* a CUDA call or kernel launch failed           */
   SHAMPOO_ENONFINITE = 4,     /* a gradient held NaN/Inf (parameter skipped)   */
   SHAMPOO_ENOTCONVERGED = 5,  /* some roots did not converge (old roots kept)  */
-  SHAMPOO_ESTATE = 6          /* call out of order (e.g. apply before roots)   */
+  SHAMPOO_ESTATE = 6,         /* call out of order (e.g. apply before roots)   */
+  SHAMPOO_EBUSY = 7           /* an asynchronous root job is still running     */
 } shampoo_status;
 
 typedef enum {
@@ -121,19 +122,70 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads);
 shampoo_status shampoo_compute_roots(shampoo_ctx* ctx);
 
 /*
+ * shampoo_compute_roots_async -- the same root computation, pipelined behind
+ * the training steps (podcast transcript, segment 16: the statistics and the
+ * preconditioned step keep running on the current roots while the next roots
+ * are computed elsewhere, then swapped in; segment 14: roots a few steps old
+ * cost next to nothing in quality).
+ *
+ * Enqueues on the context's stream a copy of the statistics as they stand
+ * after every call made so far, and returns without waiting.  A library-owned
+ * host thread then runs the coupled Newton iteration on that copy on a
+ * library-owned stream of the lowest priority, writing into a second set of
+ * roots; the roots in use are untouched until the job is installed.  The
+ * first shampoo_apply (or shampoo_install_roots) that finds the job finished
+ * swaps the new roots in; matrices that did not converge keep their previous
+ * root, as with shampoo_compute_roots.
+ *
+ * For the steps to run ahead of the root work on the GPU, give the context a
+ * stream of higher priority than the default (the library's stream has the
+ * lowest).  The second set of roots, its bf16 copy and the statistics copy
+ * (3 x 4 b^2 bytes per matrix) are allocated on the first call.
+ * Returns SHAMPOO_ESTATE before the first shampoo_update_stats, and
+ * SHAMPOO_EBUSY (nothing enqueued) while the previous job still runs; a
+ * finished, not yet installed job is installed first.
+ * While a job is in flight, shampoo_compute_roots returns SHAMPOO_EBUSY.
+ */
+shampoo_status shampoo_compute_roots_async(shampoo_ctx* ctx);
+
+/*
+ * shampoo_install_roots -- swap in the roots of a finished asynchronous job.
+ *  wait       0: install only if the job has finished; 1: block the host
+ *             until it finishes, then install.
+ *  installed  receives 1 if roots were installed by this call, else 0 (may
+ *             be NULL).
+ * Returns the job's status when it installs (SHAMPOO_OK, or
+ * SHAMPOO_ENOTCONVERGED with the counts in shampoo_root_status and
+ * shampoo_root_iterations), SHAMPOO_ECUDA if the job failed (nothing is
+ * swapped), and SHAMPOO_OK when there is nothing to install.
+ */
+shampoo_status shampoo_install_roots(shampoo_ctx* ctx, int wait, int* installed);
+
+/*
+ * shampoo_roots_generation -- how many root sets have been put in use: each
+ * shampoo_compute_roots that returns SHAMPOO_OK or SHAMPOO_ENOTCONVERGED and
+ * each install of an asynchronous job adds one.  Tells a caller at which call
+ * new roots took effect.  Host value; -1 for a NULL ctx.
+ */
+int64_t shampoo_roots_generation(const shampoo_ctx* ctx);
+
+/*
  * shampoo_apply -- precondition and update (segment 10, third piece):
  * per block P = L^{-1/p} G R^{-1/p} (per 1-D segment P = S^{-2/p} g), then
  * per parameter U = s P with the graft scale s, m <- mu m + U, W <- W - lr m.
  *  params  host array [nparams] of device float32 pointers, updated in place.
  *  grads   as for shampoo_update_stats; pass this step's gradients.
  *  lr      learning rate.
- * Returns SHAMPOO_ESTATE if roots were never computed.
+ * Returns SHAMPOO_ESTATE if roots were never computed.  First installs the
+ * roots of a finished asynchronous job, if there is one (never waits for
+ * one); a failed job's SHAMPOO_ECUDA is returned here, before any work.
  */
 shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params,
                              const void* const* grads, float lr);
 
 /*
- * shampoo_root_status -- result of the last shampoo_compute_roots.
+ * shampoo_root_status -- result of the last shampoo_compute_roots, or of
+ * the last installed asynchronous job.
  *  n_not_converged  number of matrices that kept their previous root.
  *  max_iters        largest Newton iteration count over the matrices.
  * Either pointer may be NULL.  Host values; synchronises the stream.

@@ -10,9 +10,9 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libshampoo_b200.so")
 
-OK, EINVAL, ENOMEM, ECUDA, ENONFINITE, ENOTCONVERGED, ESTATE = range(7)
+OK, EINVAL, ENOMEM, ECUDA, ENONFINITE, ENOTCONVERGED, ESTATE, EBUSY = range(8)
 STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ENOMEM", 3: "ECUDA", 4: "ENONFINITE",
-                5: "ENOTCONVERGED", 6: "ESTATE"}
+                5: "ENOTCONVERGED", 6: "ESTATE", 7: "EBUSY"}
 GRAFT_NONE, GRAFT_ADAGRAD = 0, 1
 F32, BF16 = 0, 1
 
@@ -23,6 +23,9 @@ SIGNATURES = {
                                  C.c_int, C.c_float, C.c_float, C.c_int, C.c_int, C.c_float, C.c_int, _P]),
     "shampoo_update_stats": (C.c_int, [_P, C.POINTER(_P)]),
     "shampoo_compute_roots": (C.c_int, [_P]),
+    "shampoo_compute_roots_async": (C.c_int, [_P]),
+    "shampoo_install_roots": (C.c_int, [_P, C.c_int, C.POINTER(C.c_int)]),
+    "shampoo_roots_generation": (C.c_int64, [_P]),
     "shampoo_apply": (C.c_int, [_P, C.POINTER(_P), C.POINTER(_P), C.c_float]),
     "shampoo_root_status": (C.c_int, [_P, C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "shampoo_nonfinite_status": (C.c_int, [_P, C.POINTER(C.c_int)]),
@@ -109,6 +112,22 @@ def shampoo_update_stats(ctx, grads):
 
 def shampoo_compute_roots(ctx):
     return _check(lib().shampoo_compute_roots(ctx), ctx, allow=(ENOTCONVERGED,))
+
+
+def shampoo_compute_roots_async(ctx):
+    """Queue a root job; returns EBUSY (no exception) while the previous one runs."""
+    return _check(lib().shampoo_compute_roots_async(ctx), ctx, allow=(EBUSY, ENOTCONVERGED))
+
+
+def shampoo_install_roots(ctx, wait):
+    """(status, installed) of swapping in a finished job's roots."""
+    inst = C.c_int()
+    st = _check(lib().shampoo_install_roots(ctx, int(wait), C.byref(inst)), ctx, allow=(ENOTCONVERGED,))
+    return st, inst.value
+
+
+def shampoo_roots_generation(ctx):
+    return lib().shampoo_roots_generation(ctx)
 
 
 def shampoo_apply(ctx, params, grads, lr):

@@ -7,9 +7,12 @@
 
 #include <algorithm>
 #include <cmath>
+#include <condition_variable>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
+#include <thread>
 #include <vector>
 
 #include "../../include/shampoo.h"
@@ -20,7 +23,8 @@ using namespace shampoo;
 namespace {
 
 // Per-kernel launch counts and, when enabled, CUDA-event times taken on the
-// caller's stream around each launch.
+// launching stream around each launch.  The asynchronous root thread launches
+// through the same profiler, hence the lock.
 struct Profiler {
   struct Entry {
     std::string name;
@@ -35,6 +39,7 @@ struct Profiler {
   std::vector<Entry> entries;
   std::vector<Pending> pending;
   std::vector<cudaEvent_t> pool;
+  mutable std::mutex mu;
 
   int find(const char* name) {
     for (size_t i = 0; i < entries.size(); ++i)
@@ -54,6 +59,7 @@ struct Profiler {
   }
   template <class F>
   void launch(const char* name, cudaStream_t s, F&& f) {
+    std::lock_guard<std::mutex> lock(mu);
     const int e = find(name);
     ++entries[e].launches;
     if (!on) {
@@ -67,6 +73,10 @@ struct Profiler {
     pending.push_back(Pending{e, a, b});
   }
   cudaError_t flush() {
+    std::lock_guard<std::mutex> lock(mu);
+    return flush_locked();
+  }
+  cudaError_t flush_locked() {
     cudaError_t err = cudaSuccess;
     for (auto& p : pending) {
       float ms = 0.f;
@@ -80,9 +90,21 @@ struct Profiler {
     pending.clear();
     return err;
   }
-  void reset() {
-    flush();
+  void reset(bool timing) {
+    std::lock_guard<std::mutex> lock(mu);
+    flush_locked();
     entries.clear();
+    on = timing;
+  }
+  int count() const {
+    std::lock_guard<std::mutex> lock(mu);
+    return (int)entries.size();
+  }
+  bool entry(int index, Entry* out) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (index < 0 || index >= (int)entries.size()) return false;
+    *out = entries[index];
+    return true;
   }
   ~Profiler() {
     flush();
@@ -151,9 +173,33 @@ struct shampoo_ctx {
 
   bool stats_done = false, roots_done = false;
   int last_not_converged = 0, last_max_iters = 0;
+  int64_t generation = 0;            // root sets put in use so far
   std::vector<int32_t> root_iters;   // per matrix, last compute_roots (-1-k: gave up at k)
   Profiler prof;
   std::string err;
+  int device = 0;
+
+  // Asynchronous root pipeline: a host thread runs the Newton iteration on a
+  // copy of the statistics, on its own low-priority stream, into the second
+  // set of roots; an install swaps the two sets.  `job` and the job_* results
+  // are guarded by mu; the buffers below belong to the job while it runs.
+  enum Job { kIdle, kQueued, kRunning, kDone };
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_submit = nullptr;   // recorded on `stream` after the statistics copy
+  float* stats_snap = nullptr;
+  float* roots_back = nullptr;
+  uint16_t* rplanes_back = nullptr;
+  std::thread worker;
+  std::mutex job_mu;
+  std::condition_variable cv;
+  Job job = kIdle;
+  bool quit = false;
+  shampoo_status job_status = SHAMPOO_OK;
+  std::string job_err;
+  int job_nf = 0, job_mi = 0;
+  std::vector<int32_t> job_iters;
+  double job_tol = 1e-6;   // stopping rule captured when the job was queued
+  int job_max_iters = 100;
 };
 
 namespace {
@@ -375,6 +421,117 @@ shampoo_status gather(shampoo_ctx* ctx, const void* const* grads, bool force) {
   return SHAMPOO_OK;
 }
 
+// ---------------- asynchronous root pipeline ----------------
+
+// One root job, on the root thread: Newton on the statistics copy into the
+// second set of roots, then its bf16 planes.  Errors land in `ctx`, a scratch
+// context that carries only the error text (the owner's text belongs to the
+// caller's thread).
+shampoo_status run_root_job(shampoo_ctx* o, shampoo_ctx* ctx, double tol, int max_iters, int* nf,
+                            int* mi, std::vector<int32_t>* iters) {
+  const int64_t slot = (int64_t)o->S * o->S;
+  cudaStream_t st = o->side;
+  CK(cudaStreamWaitEvent(st, o->ev_submit, 0));
+  // a matrix that does not converge keeps the root in use
+  CK(cudaMemcpyAsync(o->roots_back, o->roots, (size_t)o->nmat * slot * sizeof(float),
+                     cudaMemcpyDeviceToDevice, st));
+  shampoo_status r = run_newton(ctx, &o->prof, o->mats, o->d_mats, o->d_retry, o->stats_snap, slot, o->S, 1,
+                                o->roots_back, slot, o->S, o->S, o->eps, tol, max_iters,
+                                o->newton_chunk, o->nw, o->has_root, nullptr, o->h_count, o->ev, st, nf,
+                                mi, iters);
+  if (r != SHAMPOO_OK) {
+    cudaStreamSynchronize(st);
+    return r;
+  }
+  cudaError_t e = cudaSuccess;
+  run(&o->prof, "split_roots", st, [&] {
+    e = launch_split(o->roots_back, (int64_t)o->nmat * slot, o->rplanes_back, st);
+  });
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "split_roots");
+  CK(cudaStreamSynchronize(st));
+  return SHAMPOO_OK;
+}
+
+// The root thread: takes queued jobs one at a time until the context goes.
+void root_thread(shampoo_ctx* o) {
+  cudaSetDevice(o->device);
+  std::unique_lock<std::mutex> lock(o->job_mu);
+  for (;;) {
+    o->cv.wait(lock, [&] { return o->quit || o->job == shampoo_ctx::kQueued; });
+    if (o->quit) break;
+    o->job = shampoo_ctx::kRunning;
+    const double tol = o->job_tol;
+    const int max_iters = o->job_max_iters;
+    lock.unlock();
+    shampoo_ctx sink;
+    int nf = 0, mi = 0;
+    std::vector<int32_t> it;
+    shampoo_status r = run_root_job(o, &sink, tol, max_iters, &nf, &mi, &it);
+    if (r == SHAMPOO_OK && nf) r = SHAMPOO_ENOTCONVERGED;
+    lock.lock();
+    o->job_status = r;
+    o->job_err = r == SHAMPOO_ENOTCONVERGED ? std::to_string(nf) + " roots did not converge" : sink.err;
+    o->job_nf = nf;
+    o->job_mi = mi;
+    o->job_iters.swap(it);
+    o->job = shampoo_ctx::kDone;
+    o->cv.notify_all();
+  }
+}
+
+// Swap in the roots of a finished job; with `wait`, first block until the
+// job in flight (if any) finishes.
+shampoo_status install_roots(shampoo_ctx* ctx, bool wait, int* installed) {
+  if (installed) *installed = 0;
+  std::unique_lock<std::mutex> lock(ctx->job_mu);
+  if (wait)
+    ctx->cv.wait(lock, [&] { return ctx->job != shampoo_ctx::kQueued && ctx->job != shampoo_ctx::kRunning; });
+  if (ctx->job != shampoo_ctx::kDone) return SHAMPOO_OK;
+  ctx->job = shampoo_ctx::kIdle;
+  const shampoo_status r = ctx->job_status;
+  if (r != SHAMPOO_OK && r != SHAMPOO_ENOTCONVERGED)
+    return fail(ctx, r, "asynchronous root job failed: " + ctx->job_err);
+  std::swap(ctx->roots, ctx->roots_back);
+  std::swap(ctx->rplanes, ctx->rplanes_back);
+  if (!ctx->blocks.empty() &&
+      !encode_planes(&ctx->maps.rk, ctx->rplanes, ctx->S, 2 * (int64_t)ctx->nmat, 64, 128))
+    return fail(ctx, SHAMPOO_ECUDA, "cuTensorMapEncodeTiled failed");
+  ctx->roots_done = true;
+  ctx->last_not_converged = ctx->job_nf;
+  ctx->last_max_iters = ctx->job_mi;
+  ctx->root_iters = ctx->job_iters;
+  ++ctx->generation;
+  if (installed) *installed = 1;
+  if (r == SHAMPOO_ENOTCONVERGED) return fail(ctx, r, ctx->job_err);
+  return SHAMPOO_OK;
+}
+
+bool job_in_flight(shampoo_ctx* ctx) {
+  std::lock_guard<std::mutex> lock(ctx->job_mu);
+  return ctx->job == shampoo_ctx::kQueued || ctx->job == shampoo_ctx::kRunning;
+}
+
+// First asynchronous call: the second set of buffers, the low-priority
+// stream and the root thread.
+shampoo_status start_pipeline(shampoo_ctx* ctx) {
+  const size_t n = (size_t)ctx->nmat * ctx->S * ctx->S;
+  cudaError_t e = cudaSuccess;
+  float *snap = nullptr, *back = nullptr;
+  uint16_t* planes = nullptr;
+  if ((e = dalloc(ctx, &snap, n)) != cudaSuccess || (e = dalloc(ctx, &back, n)) != cudaSuccess ||
+      (e = dalloc(ctx, &planes, 2 * n)) != cudaSuccess)
+    return fail(ctx, SHAMPOO_ENOMEM, std::string("asynchronous root buffers: ") + cudaGetErrorString(e));
+  int least = 0, greatest = 0;
+  CK(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+  CK(cudaStreamCreateWithPriority(&ctx->side, cudaStreamNonBlocking, least));
+  CK(cudaEventCreateWithFlags(&ctx->ev_submit, cudaEventDisableTiming));
+  ctx->stats_snap = snap;
+  ctx->roots_back = back;
+  ctx->rplanes_back = planes;
+  ctx->worker = std::thread(root_thread, ctx);
+  return SHAMPOO_OK;
+}
+
 }  // namespace
 
 namespace shampoo {
@@ -393,6 +550,19 @@ const char* shampoo_last_error(const shampoo_ctx* ctx) {
 
 void shampoo_destroy(shampoo_ctx* ctx) {
   if (!ctx) return;
+  if (ctx->worker.joinable()) {   // a running root job finishes first; a queued one is dropped
+    {
+      std::lock_guard<std::mutex> lock(ctx->job_mu);
+      ctx->quit = true;
+    }
+    ctx->cv.notify_all();
+    ctx->worker.join();
+  }
+  if (ctx->side) {
+    cudaStreamSynchronize(ctx->side);
+    cudaStreamDestroy(ctx->side);
+  }
+  if (ctx->ev_submit) cudaEventDestroy(ctx->ev_submit);
   cudaStreamSynchronize(ctx->stream);
   for (void* q : ctx->allocs) cudaFree(q);
   if (ctx->h_count) cudaFreeHost(ctx->h_count);
@@ -421,6 +591,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
 
   shampoo_ctx* ctx = new shampoo_ctx();
   ctx->stream = static_cast<cudaStream_t>(cuda_stream);
+  cudaGetDevice(&ctx->device);
   ctx->nparams = nparams;
   ctx->b = ctx->S = block_size;
   ctx->p = p;
@@ -607,6 +778,11 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   int nf = 0, mi = 0;
   if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots before update_stats");
+  if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "an asynchronous root job is in flight");
+  {   // a finished job's roots are older than these: install, then overwrite
+    const shampoo_status ir = install_roots(ctx, false, nullptr);
+    if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
+  }
   const int64_t slot = (int64_t)ctx->S * ctx->S;
   shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->d_retry, ctx->stats,
                                  slot, ctx->S, 1,
@@ -620,15 +796,51 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
   });
   if (e != cudaSuccess) return cuda_fail(ctx, e, "split_roots");
   ctx->roots_done = true;
+  ++ctx->generation;
   ctx->last_not_converged = nf;
   ctx->last_max_iters = mi;
   if (nf) return fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
   return SHAMPOO_OK;
 }
 
+shampoo_status shampoo_compute_roots_async(shampoo_ctx* ctx) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots_async before update_stats");
+  if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "the previous asynchronous root job is still running");
+  const shampoo_status ir = install_roots(ctx, false, nullptr);
+  if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
+  if (!ctx->worker.joinable()) {
+    const shampoo_status ps = start_pipeline(ctx);
+    if (ps != SHAMPOO_OK) return ps;
+  }
+  // the statistics as they stand after every call so far
+  const size_t n = (size_t)ctx->nmat * ctx->S * ctx->S;
+  CK(cudaMemcpyAsync(ctx->stats_snap, ctx->stats, n * sizeof(float), cudaMemcpyDeviceToDevice, ctx->stream));
+  CK(cudaEventRecord(ctx->ev_submit, ctx->stream));
+  {
+    std::lock_guard<std::mutex> lock(ctx->job_mu);
+    ctx->job_tol = ctx->tol;
+    ctx->job_max_iters = ctx->max_iters;
+    ctx->job = shampoo_ctx::kQueued;
+  }
+  ctx->cv.notify_all();
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_install_roots(shampoo_ctx* ctx, int wait, int* installed) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  return install_roots(ctx, wait != 0, installed);
+}
+
+int64_t shampoo_roots_generation(const shampoo_ctx* ctx) { return ctx ? ctx->generation : -1; }
+
 shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void* const* grads,
                              float lr) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  {
+    const shampoo_status ir = install_roots(ctx, false, nullptr);
+    if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
+  }
   if (!ctx->roots_done) return fail(ctx, SHAMPOO_ESTATE, "apply before compute_roots");
   if (!params) return fail(ctx, SHAMPOO_EINVAL, "params is NULL");
   shampoo_status st = set_pointers(ctx, grads, params);
@@ -746,20 +958,18 @@ shampoo_status shampoo_root_iterations(shampoo_ctx* ctx, int32_t* out) {
 
 shampoo_status shampoo_profile_enable(shampoo_ctx* ctx, int on) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
-  ctx->prof.reset();
-  ctx->prof.on = on != 0;
+  ctx->prof.reset(on != 0);
   return SHAMPOO_OK;
 }
 
-int shampoo_profile_count(const shampoo_ctx* ctx) { return ctx ? (int)ctx->prof.entries.size() : 0; }
+int shampoo_profile_count(const shampoo_ctx* ctx) { return ctx ? ctx->prof.count() : 0; }
 
 shampoo_status shampoo_profile_entry(shampoo_ctx* ctx, int index, char* name, int name_len,
                                      int64_t* launches, double* ms) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   CK(ctx->prof.flush());
-  if (index < 0 || index >= (int)ctx->prof.entries.size())
-    return fail(ctx, SHAMPOO_EINVAL, "profile index out of range");
-  const auto& e = ctx->prof.entries[index];
+  Profiler::Entry e;
+  if (!ctx->prof.entry(index, &e)) return fail(ctx, SHAMPOO_EINVAL, "profile index out of range");
   if (name && name_len > 0) {
     std::strncpy(name, e.name.c_str(), name_len - 1);
     name[name_len - 1] = 0;

@@ -43,6 +43,20 @@ class Shampoo:
         """Returns True when every root converged."""
         return L.shampoo_compute_roots(self.ctx) == L.OK
 
+    def compute_roots_async(self):
+        """Queue a root job on the library's low-priority stream and return at
+        once.  Returns False (nothing queued) while the previous job runs."""
+        return L.shampoo_compute_roots_async(self.ctx) != L.EBUSY
+
+    def install_roots(self, wait=False):
+        """Swap in a finished job's roots (blocking for it with wait=True).
+        Returns True when roots were installed."""
+        return L.shampoo_install_roots(self.ctx, wait)[1] == 1
+
+    def roots_generation(self):
+        """Root sets put in use so far (sync computes and async installs)."""
+        return L.shampoo_roots_generation(self.ctx)
+
     def apply(self, params, grads, lr):
         self._check_tensors(params, "params")
         self._check_tensors(grads, "grads")

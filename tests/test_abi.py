@@ -81,6 +81,9 @@ def test_null_context_calls(lib):
     assert lib.shampoo_compute_roots(None) == L.EINVAL
     assert lib.shampoo_apply(None, None, None, 0.1) == L.EINVAL
     assert lib.shampoo_num_matrices(None) == 0
+    assert lib.shampoo_compute_roots_async(None) == L.EINVAL
+    assert lib.shampoo_install_roots(None, 0, None) == L.EINVAL
+    assert lib.shampoo_roots_generation(None) == -1
     lib.shampoo_destroy(None)
 
 

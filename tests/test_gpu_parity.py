@@ -324,3 +324,112 @@ def test_resnet50_full_set():
     c = wl.CONFIGS["resnet50_b128"]
     w = run_subset(c, steps=3, interval=2, keep=list(range(len(c["shapes"]))))
     assert w["dW"] <= STEP_TOL and w["W"] <= STEP_TOL, w
+
+
+# --------------------------------------------------------------------------
+# asynchronous roots (podcast transcript, segment 16): the steps keep using
+# the roots in place while the next ones are computed, then swap them in
+# --------------------------------------------------------------------------
+def run_async_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, submit, wait_at, seed, gstd):
+    """Roots synchronously at step 0; an asynchronous job queued after the
+    statistics of each step in `submit`; a blocking install before the apply
+    of each step in `wait_at`.  The library swaps a finished job in at an
+    apply of its choosing; the test reads at which one from the roots
+    generation and installs, on the oracle, the roots of the statistics as
+    they stood at submission before the same step's apply."""
+    import copy
+    from shampoo_second_order_b200 import Shampoo
+    o = ShampooOracle(shapes, b, beta2, eps, 4, graft, mu)
+    opt = Shampoo(shapes, b, beta2, eps, 4, graft, mu, gdtype)
+    W0 = wl.make_params(shapes, seed)
+    Wo = [w.astype(np.float64) for w in W0]
+    Wd = [torch.from_numpy(w).cuda() for w in W0]
+    worst = {"dW": 0.0, "W": 0.0}
+    pending = None
+    installs = []
+    for t in range(steps):
+        g = wl.make_grads(shapes, seed, t, gstd, gdtype)
+        gd = [to_dev(x, gdtype) for x in g]
+        prev_d = [w.cpu().numpy().astype(np.float64) for w in Wd]
+        prev_o = Wo
+        o.update_stats(g)
+        opt.update_stats(gd)
+        if t == 0:
+            o.compute_roots()
+            opt.compute_roots()
+        if t in submit:
+            kept = list(o.roots)          # compute_roots replaces the entries of o.roots
+            o.compute_roots()
+            pending, o.roots = o.roots, kept
+            assert opt.compute_roots_async()
+        gen0 = opt.roots_generation()
+        if t in wait_at:
+            opt.install_roots(wait=True)
+        opt.apply(Wd, gd, lr)
+        if opt.roots_generation() > gen0:
+            assert pending is not None
+            o.roots, pending = copy.deepcopy(pending), None
+            installs.append(t)
+        Wo = o.apply(Wo, g, lr)
+        torch.cuda.synchronize()
+        for i, s in enumerate(shapes):
+            wd = Wd[i].cpu().numpy().astype(np.float64)
+            for sl in pieces(s, b):
+                worst["dW"] = max(worst["dW"], rel((wd - prev_d[i])[sl], (Wo[i] - prev_o[i])[sl]))
+                worst["W"] = max(worst["W"], rel(wd[sl], Wo[i][sl]))
+    assert pending is None
+    opt.close()
+    return worst, installs
+
+
+@pytest.mark.parametrize("gdtype", ["f32", "bf16"])
+def test_async_roots_ragged_set(gdtype):
+    shapes = [(200, 130), (64, 64), (19, 200), (130,), (64,), (1, 77)]
+    w, installs = run_async_pair(shapes, 64, 0.99, 1e-6, 1, 0.0, 0.1, gdtype, steps=9,
+                                 submit=(2, 5), wait_at=(4, 8), seed=7, gstd=1e-2)
+    assert w["dW"] <= STEP_TOL and w["W"] <= STEP_TOL, w
+    assert len(installs) == 2 and 2 <= installs[0] <= 4 and 5 <= installs[1] <= 8, installs
+
+
+def test_async_roots_transformer_layer_b512():
+    """The bench's set and launch configuration: roots at step 0, an
+    asynchronous job after step 20's statistics, installed by step 24."""
+    c = wl.CONFIGS["transformer_layer_b512"]
+    w, installs = run_async_pair(c["shapes"], c["block_size"], c["beta2"], c["eps"], c["graft"],
+                                 c["momentum"], c["lr"], c["grad_dtype"], steps=25, submit=(20,),
+                                 wait_at=(24,), seed=c["seed"], gstd=c["grad_std"])
+    assert w["dW"] <= STEP_TOL and w["W"] <= STEP_TOL, w
+    assert len(installs) == 1 and 20 <= installs[0] <= 24, installs
+
+
+def test_async_roots_busy_and_sync_refused():
+    """While a job runs, a second submission and a synchronous computation
+    are refused with EBUSY and leave the roots in use untouched; after the
+    install the new roots equal the synchronous ones of the same statistics."""
+    from shampoo_second_order_b200 import Shampoo, _lib
+    c = wl.CONFIGS["transformer_layer_b512"]
+    shapes = c["shapes"]
+    opt = Shampoo(shapes, c["block_size"], c["beta2"], c["eps"], 4, 1, 0.0, "bf16")
+    g = [to_dev(x, "bf16") for x in wl.make_grads(shapes, 3, 0, 1e-3, "bf16")]
+    opt.update_stats(g)
+    opt.compute_roots()
+    X_sync0, _ = opt.read_matrix(1, 0)
+    g = [to_dev(x, "bf16") for x in wl.make_grads(shapes, 3, 1, 1e-3, "bf16")]
+    opt.update_stats(g)
+    gen = opt.roots_generation()
+    assert opt.compute_roots_async()
+    busy = not opt.compute_roots_async()          # about ten milliseconds of Newton work queued
+    if busy:
+        with pytest.raises(_lib.ShampooError) as e:
+            opt.compute_roots()
+        assert e.value.status == _lib.EBUSY
+    X_now, _ = opt.read_matrix(1, 0)
+    if opt.roots_generation() == gen:
+        assert np.array_equal(X_now, X_sync0)
+    assert opt.install_roots(wait=True) or opt.roots_generation() == gen + 1
+    X_async, _ = opt.read_matrix(1, 0)
+    opt.compute_roots()                           # the same statistics, synchronously
+    X_sync1, _ = opt.read_matrix(1, 0)
+    assert rel(X_async, X_sync1) <= 1e-6
+    assert busy
+    opt.close()
