@@ -95,6 +95,24 @@ def newton_flops(cfg, iters, per_kernel=False):
     return (a, b, c) if per_kernel else a + b + c
 
 
+def ozaki_ops(cfg, iters, slices, per_kernel=False):
+    """int8 tensor-core operations the emulated Newton products execute: per
+    product, every 128 x 64 tile of the upper triangle of the b x b slot runs
+    slices (slices + 1) / 2 digit products over the padded K = b."""
+    S = -(-cfg["block_size"] // 64) * 64
+    tc, tr = S // 64, -(-S // 128)
+    ntri = sum(max(0, tc - 2 * ti) for ti in range(tr))
+    nk = -(-S // 128)
+    per = ntri * nk * 128 * 2 * 128 * 64 * slices * (slices + 1) // 2
+    a = b = c = 0
+    for (n, prods), k in zip(matrix_sizes(cfg), iters):
+        k = k if k >= 0 else -1 - k
+        a += 2 * k * per
+        b += (k * per) if prods == 4 else 0
+        c += k * per
+    return (a, b, c) if per_kernel else a + b + c
+
+
 def numel(cfg):
     return wl.count_params(cfg["shapes"])
 
@@ -233,7 +251,7 @@ def tc_work(cfg, kernel):
     return fl, by
 
 
-def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak):
+def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak, slices=6):
     """Achieved vs peak for the kernel with the largest share of device time."""
     names = {k: v for k, v in prof.items() if v[1] > 0}
     if not names:
@@ -252,6 +270,11 @@ def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak):
         fl = {"newton_step_a": a, "newton_step_b": b, "newton_step_c": c}[top]
         work = ("tensor", fl / 1e12 / sec, fp64_peak, "TFLOP/s", fl / max(launches, 1),
                 "cuBLAS DGEMM (fp64) measured in this run")
+    elif top.startswith("ozaki_step"):
+        a, b, c = ozaki_ops(cfg, iters_sum, slices, per_kernel=True)
+        ops = {"ozaki_step_a": a, "ozaki_step_b": b, "ozaki_step_c": c}[top]
+        work = ("tensor", ops / 1e12 / sec, 2 * bf16, "TOP/s", ops / max(launches, 1),
+                "MEASURED_PEAKS.json bf16_tflops (burst) x 2, the int8 : bf16 dense ratio")
     elif top in ("stats_tc", "apply_y_tc", "apply_p_tc"):
         fl, by = tc_work(cfg, top)
         fl, by = fl * launches, by * launches
@@ -401,7 +424,8 @@ def roots_bench(args):
             s.record(stream)
             its = []
             for p in c["ps"]:
-                X, it = batched_inverse_root(dA, p, c["eps"], c["tol"], stream=stream)
+                X, it = batched_inverse_root(dA, p, c["eps"], c["tol"], stream=stream, method=args.roots,
+                                             slices=args.slices)
                 its.append((p, it))
             e.record(stream)
         stream.synchronize()
@@ -417,7 +441,9 @@ def roots_bench(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "batched_roots_512", "batch": batch, "n": n, "p": list(c["ps"]),
-                       "tol": c["tol"], "l2": "flushed between steps (256 MiB write)"},
+                       "tol": c["tol"], "l2": "flushed between steps (256 MiB write)",
+                       "newton_products": (args.roots if args.roots == "fp64"
+                                           else f"int8-emulated fp64, {args.slices} slices")},
             "roofline": {"kernel": "newton (all launches of one call)", "bound": "tensor",
                          "achieved": round(val, 3), "peak": round(fp64_peak, 2), "unit": "TFLOP/s",
                          "frac": round(val / fp64_peak, 4), "traffic": None,
@@ -442,6 +468,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-async", action="store_true")
+    ap.add_argument("--roots", default="fp64", choices=["fp64", "int8"],
+                    help="Newton products in float64 or emulated on the int8 tensor cores")
+    ap.add_argument("--slices", type=int, default=6)
     args = ap.parse_args()
     if args.config == "batched_roots_512":
         return roots_bench(args)
@@ -494,6 +523,7 @@ def main():
 
     opt = Shampoo(shapes, cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"], cfg["graft"],
                   cfg["momentum"], cfg["grad_dtype"], stream=stream)
+    opt.set_root_method(args.roots, args.slices)
     lr = cfg["lr"]
     interval = cfg["root_interval"]
 
@@ -643,7 +673,7 @@ def main():
                       "sync_step_ms_max": max(s_.elapsed_time(e_) for s_, e_ in ev),
                       "streams": "steps at high priority; roots on the library's lowest-priority stream"}
 
-    top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak)
+    top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak, args.slices)
 
     if rank == 0:
         phase = {}
@@ -667,6 +697,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
             "config": {"workload": args.config, "params": numel(cfg), "block_size": cfg["block_size"],
                        "grad_dtype": cfg["grad_dtype"], "root_interval": interval,
+                       "newton_products": (args.roots if args.roots == "fp64"
+                                           else f"int8-emulated fp64, {args.slices} slices"),
                        "root_steps_timed": n_root, "l2": "flushed between steps (256 MiB write)",
                        "parallelism": f"replicas x{world}"},
             "roofline": roof, "cpu_baseline": cpu_line, "e2e": e2e, "async_roots": async_line,

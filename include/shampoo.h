@@ -60,6 +60,12 @@ typedef enum {
 } shampoo_graft;
 
 typedef enum {
+  SHAMPOO_ROOTS_FP64 = 0,          /* Newton products in float64 (mma f64)     */
+  SHAMPOO_ROOTS_INT8_EMULATED = 1  /* the same products emulated on the int8
+                                      tensor cores (Ozaki scheme)              */
+} shampoo_root_method;
+
+typedef enum {
   SHAMPOO_F32 = 0,            /* gradients are float32                         */
   SHAMPOO_BF16 = 1            /* gradients are bfloat16 (statistics in fp32)   */
 } shampoo_dtype;
@@ -206,6 +212,25 @@ shampoo_status shampoo_nonfinite_status(shampoo_ctx* ctx, int* n_params_skipped)
 shampoo_status shampoo_set_root_options(shampoo_ctx* ctx, double tol, int max_iters);
 
 /*
+ * shampoo_set_root_method -- how later root calls multiply matrices inside
+ * the coupled Newton iteration (the iteration, its stopping rule and its
+ * float64 state are the same for both).
+ *  method  SHAMPOO_ROOTS_FP64: float64 products (the default).
+ *          SHAMPOO_ROOTS_INT8_EMULATED: each float64 operand row is cut into
+ *          `slices` signed 7-bit digits below a per-row power of two, and a
+ *          product is the exact int32 sum of the digit products whose weights
+ *          reach 2^{-7 (slices+1)} (Ozaki scheme), run on the int8 tensor
+ *          cores.  Per entry the error is of order n 2^{-7 slices} times the
+ *          row and column scales (2^-42 n for 6 slices), against 2^-53 for a
+ *          float64 product.
+ *  slices  4..7 for the emulated method (6 recommended); ignored otherwise.
+ * The emulated method allocates 35 int8 planes of b x b bytes (5 iterates x 7
+ * slices) per matrix of a Newton chunk on first use.  SHAMPOO_EBUSY while an
+ * asynchronous root job runs.
+ */
+shampoo_status shampoo_set_root_method(shampoo_ctx* ctx, int method, int slices);
+
+/*
  * shampoo_num_matrices -- number of statistics matrices: 2 per 2-D block
  * (L then R, blocks in parameter order, row-major within a parameter), then
  * 1 per 1-D segment (parameter order).  Each lives in a b x b slot.
@@ -284,6 +309,17 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
                                             int n, int p, float eps, double tol,
                                             int max_iters, int32_t* iters,
                                             void* stream);
+
+/*
+ * shampoo_batched_inverse_root_ex -- shampoo_batched_inverse_root with the
+ * product method of shampoo_set_root_method (method, slices).  The emulated
+ * method also allocates its int8 slice planes (35 n' x n' bytes per matrix in
+ * flight, n' = n rounded up to 64) and frees them before returning.
+ */
+shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int batch,
+                                               int n, int p, float eps, double tol,
+                                               int max_iters, int32_t* iters,
+                                               void* stream, int method, int slices);
 
 /*
  * shampoo_batched_inverse_root_noalloc -- shampoo_batched_inverse_root for

@@ -14,6 +14,7 @@ OK, EINVAL, ENOMEM, ECUDA, ENONFINITE, ENOTCONVERGED, ESTATE, EBUSY = range(8)
 STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ENOMEM", 3: "ECUDA", 4: "ENONFINITE",
                 5: "ENOTCONVERGED", 6: "ESTATE", 7: "EBUSY"}
 GRAFT_NONE, GRAFT_ADAGRAD = 0, 1
+ROOTS_FP64, ROOTS_INT8_EMULATED = 0, 1
 F32, BF16 = 0, 1
 
 # name -> (restype, argtypes), exactly the declarations of include/shampoo.h
@@ -30,6 +31,7 @@ SIGNATURES = {
     "shampoo_root_status": (C.c_int, [_P, C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "shampoo_nonfinite_status": (C.c_int, [_P, C.POINTER(C.c_int)]),
     "shampoo_set_root_options": (C.c_int, [_P, C.c_double, C.c_int]),
+    "shampoo_set_root_method": (C.c_int, [_P, C.c_int, C.c_int]),
     "shampoo_num_matrices": (C.c_int, [_P]),
     "shampoo_matrix_info": (C.c_int, [_P, C.c_int, C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "shampoo_read_matrix": (C.c_int, [_P, C.c_int, C.c_int, _P]),
@@ -42,6 +44,8 @@ SIGNATURES = {
     "shampoo_destroy": (None, [_P]),
     "shampoo_batched_inverse_root": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_float,
                                                C.c_double, C.c_int, _P, _P]),
+    "shampoo_batched_inverse_root_ex": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_float,
+                                                  C.c_double, C.c_int, _P, _P, C.c_int, C.c_int]),
     "shampoo_batched_inverse_root_noalloc": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_float,
                                                        C.c_double, C.c_int, _P, _P]),
     "shampoo_version": (C.c_char_p, []),
@@ -150,6 +154,10 @@ def shampoo_set_root_options(ctx, tol, max_iters):
     return _check(lib().shampoo_set_root_options(ctx, float(tol), int(max_iters)), ctx)
 
 
+def shampoo_set_root_method(ctx, method, slices=6):
+    return _check(lib().shampoo_set_root_method(ctx, int(method), int(slices)), ctx)
+
+
 def shampoo_num_matrices(ctx):
     return lib().shampoo_num_matrices(ctx)
 
@@ -196,6 +204,15 @@ def shampoo_batched_inverse_root(A_ptr, X_ptr, batch, n, p, eps, tol, max_iters,
                                             int(batch), int(n), int(p), float(eps), float(tol),
                                             int(max_iters), C.c_void_p(int(iters_ptr)),
                                             C.c_void_p(int(stream)))
+    return _check(st, None, allow=(ENOTCONVERGED,))
+
+
+def shampoo_batched_inverse_root_ex(A_ptr, X_ptr, batch, n, p, eps, tol, max_iters, iters_ptr=0,
+                                    stream=0, method=ROOTS_FP64, slices=6):
+    st = lib().shampoo_batched_inverse_root_ex(C.c_void_p(int(A_ptr)), C.c_void_p(int(X_ptr)),
+                                               int(batch), int(n), int(p), float(eps), float(tol),
+                                               int(max_iters), C.c_void_p(int(iters_ptr)),
+                                               C.c_void_p(int(stream)), int(method), int(slices))
     return _check(st, None, allow=(ENOTCONVERGED,))
 
 

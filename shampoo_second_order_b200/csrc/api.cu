@@ -167,6 +167,9 @@ struct shampoo_ctx {
   NewtonWork nw{};
   NewtonMat* d_retry = nullptr;
   int newton_chunk = 0;
+  int root_method = SHAMPOO_ROOTS_FP64;   // or SHAMPOO_ROOTS_INT8_EMULATED
+  int oz_slices = 6;
+  OzakiMaps oz{};                          // over nw.q, once allocated
   int* h_count = nullptr;   // pinned [2]
   cudaEvent_t ev[2] = {nullptr, nullptr};
   std::vector<void*> allocs;
@@ -198,8 +201,9 @@ struct shampoo_ctx {
   std::string job_err;
   int job_nf = 0, job_mi = 0;
   std::vector<int32_t> job_iters;
-  double job_tol = 1e-6;   // stopping rule captured when the job was queued
+  double job_tol = 1e-6;   // stopping rule and product method captured when the job was queued
   int job_max_iters = 100;
+  bool job_oz = false;
 };
 
 namespace {
@@ -279,7 +283,8 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
                           float eps, double tol, int max_iters, int chunk, NewtonWork& w,
                           int* has_root, int32_t* iters_out, int* h_count, cudaEvent_t* ev,
                           cudaStream_t st, int* n_failed, int* max_it,
-                          std::vector<int32_t>* per_slot) {
+                          std::vector<int32_t>* per_slot, const OzakiMaps* oz = nullptr,
+                          int* oz_err = nullptr) {
   *n_failed = 0;
   *max_it = 0;
   const int nm_all = (int)hm.size();
@@ -302,14 +307,35 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
       run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, upper, d, nm, S, w, st); });
       run(pr, "newton_lanczos", st, [&] { launch_newton_lanczos(d, nm, S, w, st); });
       run(pr, "newton_t0", st, [&] { launch_newton_t0(d, nm, S, w, st); });
+      cudaError_t oe = cudaSuccess;
+      if (oz)
+        run(pr, "ozaki_split", st, [&] {
+          oe = launch_ozaki_split(d, nm, S, 0, (1u << kOzX) | (1u << kOzT) | (1u << kOzM), w, st);
+        });
       run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
       CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
       CK(cudaEventRecord(ev[0], st));
       for (int it = 0; it < max_iters; ++it) {
         // the check of M_it is in flight; queue step it+1 before waiting for it
-        run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, w, st); });
-        if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, w, st); });
-        run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, w, st); });
+        if (oz) {   // the same step with emulated float64 products on the int8 tensor cores
+          run(pr, "ozaki_step_a", st, [&] { oe = launch_ozaki_step(*oz, 0, d, nm, S, it, w, oz_err, st); });
+          run(pr, "ozaki_split", st, [&] {
+            oe = launch_ozaki_split(d, nm, S, it + 1, (1u << kOzX) | (1u << kOzT2), w, st);
+          });
+          if (has_p4) {
+            run(pr, "ozaki_step_b", st, [&] { oe = launch_ozaki_step(*oz, 1, d, nm, S, it, w, oz_err, st); });
+            run(pr, "ozaki_split", st, [&] { oe = launch_ozaki_split(d, nm, S, it + 1, 1u << kOzT4, w, st); });
+          }
+          run(pr, "ozaki_step_c", st, [&] { oe = launch_ozaki_step(*oz, 2, d, nm, S, it, w, oz_err, st); });
+          run(pr, "ozaki_split", st, [&] {
+            oe = launch_ozaki_split(d, nm, S, it + 1, (1u << kOzM) | (1u << kOzT), w, st);
+          });
+          if (oe != cudaSuccess) return cuda_fail(ctx, oe, "emulated Newton step");
+        } else {
+          run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, w, st); });
+          if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, w, st); });
+          run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, w, st); });
+        }
         run(pr, "newton_check", st, [&] { launch_newton_check(nm, it + 1, tol, max_iters, w, st); });
         const int nx = (it + 1) & 1;
         CK(cudaGetLastError());
@@ -421,14 +447,44 @@ shampoo_status gather(shampoo_ctx* ctx, const void* const* grads, bool force) {
   return SHAMPOO_OK;
 }
 
+// Slice planes of the emulated products, allocated on first use: room for
+// kOzMaxSlices slices of kOzSets iterates of every matrix of a Newton chunk.
+shampoo_status ensure_ozaki(shampoo_ctx* ctx) {
+  if (ctx->nw.q) return SHAMPOO_OK;
+  const int S = ctx->S, cap = ctx->newton_chunk;
+  const int64_t planes = (int64_t)kOzSets * kOzMaxSlices * cap;
+  int8_t* q = nullptr;
+  int* qe = nullptr;
+  cudaError_t e = dalloc(ctx, &q, (size_t)planes * S * S);
+  if (e == cudaSuccess) e = dalloc(ctx, &qe, (size_t)kOzSets * cap * S);
+  if (e != cudaSuccess) return fail(ctx, SHAMPOO_ENOMEM, std::string("int8 slice planes: ") + cudaGetErrorString(e));
+  auto fn = encode_fn();
+  cuuint64_t dims[3] = {(cuuint64_t)S, (cuuint64_t)S, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)S, (cuuint64_t)S * S};
+  cuuint32_t box_a[3] = {128, 128, 1}, box_b[3] = {128, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  if (!fn ||
+      fn(&ctx->oz.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box_a, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      fn(&ctx->oz.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box_b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return fail(ctx, SHAMPOO_ECUDA, "cuTensorMapEncodeTiled failed for the slice planes");
+  ctx->nw.q = q;
+  ctx->nw.qe = qe;
+  ctx->nw.qcap = cap;
+  return SHAMPOO_OK;
+}
+
 // ---------------- asynchronous root pipeline ----------------
 
 // One root job, on the root thread: Newton on the statistics copy into the
 // second set of roots, then its bf16 planes.  Errors land in `ctx`, a scratch
 // context that carries only the error text (the owner's text belongs to the
 // caller's thread).
-shampoo_status run_root_job(shampoo_ctx* o, shampoo_ctx* ctx, double tol, int max_iters, int* nf,
-                            int* mi, std::vector<int32_t>* iters) {
+shampoo_status run_root_job(shampoo_ctx* o, shampoo_ctx* ctx, double tol, int max_iters, bool use_oz,
+                            int* nf, int* mi, std::vector<int32_t>* iters) {
   const int64_t slot = (int64_t)o->S * o->S;
   cudaStream_t st = o->side;
   CK(cudaStreamWaitEvent(st, o->ev_submit, 0));
@@ -438,7 +494,7 @@ shampoo_status run_root_job(shampoo_ctx* o, shampoo_ctx* ctx, double tol, int ma
   shampoo_status r = run_newton(ctx, &o->prof, o->mats, o->d_mats, o->d_retry, o->stats_snap, slot, o->S, 1,
                                 o->roots_back, slot, o->S, o->S, o->eps, tol, max_iters,
                                 o->newton_chunk, o->nw, o->has_root, nullptr, o->h_count, o->ev, st, nf,
-                                mi, iters);
+                                mi, iters, use_oz ? &o->oz : nullptr, o->d_err);
   if (r != SHAMPOO_OK) {
     cudaStreamSynchronize(st);
     return r;
@@ -462,11 +518,12 @@ void root_thread(shampoo_ctx* o) {
     o->job = shampoo_ctx::kRunning;
     const double tol = o->job_tol;
     const int max_iters = o->job_max_iters;
+    const bool use_oz = o->job_oz;
     lock.unlock();
     shampoo_ctx sink;
     int nf = 0, mi = 0;
     std::vector<int32_t> it;
-    shampoo_status r = run_root_job(o, &sink, tol, max_iters, &nf, &mi, &it);
+    shampoo_status r = run_root_job(o, &sink, tol, max_iters, use_oz, &nf, &mi, &it);
     if (r == SHAMPOO_OK && nf) r = SHAMPOO_ENOTCONVERGED;
     lock.lock();
     o->job_status = r;
@@ -784,11 +841,18 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
     if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
   }
   const int64_t slot = (int64_t)ctx->S * ctx->S;
+  const bool use_oz = ctx->root_method == SHAMPOO_ROOTS_INT8_EMULATED;
+  if (use_oz) {
+    const shampoo_status os = ensure_ozaki(ctx);
+    if (os != SHAMPOO_OK) return os;
+    ctx->nw.qs = ctx->oz_slices;
+  }
   shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->d_retry, ctx->stats,
                                  slot, ctx->S, 1,
                                  ctx->roots, slot, ctx->S, ctx->S, ctx->eps, ctx->tol,
                                  ctx->max_iters, ctx->newton_chunk, ctx->nw, ctx->has_root, nullptr,
-                                 ctx->h_count, ctx->ev, ctx->stream, &nf, &mi, &ctx->root_iters);
+                                 ctx->h_count, ctx->ev, ctx->stream, &nf, &mi, &ctx->root_iters,
+                                 use_oz ? &ctx->oz : nullptr, ctx->d_err);
   if (st != SHAMPOO_OK) return st;
   cudaError_t e = cudaSuccess;
   run(&ctx->prof, "split_roots", ctx->stream, [&] {
@@ -813,6 +877,12 @@ shampoo_status shampoo_compute_roots_async(shampoo_ctx* ctx) {
     const shampoo_status ps = start_pipeline(ctx);
     if (ps != SHAMPOO_OK) return ps;
   }
+  const bool use_oz = ctx->root_method == SHAMPOO_ROOTS_INT8_EMULATED;
+  if (use_oz) {
+    const shampoo_status os = ensure_ozaki(ctx);
+    if (os != SHAMPOO_OK) return os;
+    ctx->nw.qs = ctx->oz_slices;
+  }
   // the statistics as they stand after every call so far
   const size_t n = (size_t)ctx->nmat * ctx->S * ctx->S;
   CK(cudaMemcpyAsync(ctx->stats_snap, ctx->stats, n * sizeof(float), cudaMemcpyDeviceToDevice, ctx->stream));
@@ -821,6 +891,7 @@ shampoo_status shampoo_compute_roots_async(shampoo_ctx* ctx) {
     std::lock_guard<std::mutex> lock(ctx->job_mu);
     ctx->job_tol = ctx->tol;
     ctx->job_max_iters = ctx->max_iters;
+    ctx->job_oz = use_oz;
     ctx->job = shampoo_ctx::kQueued;
   }
   ctx->cv.notify_all();
@@ -920,6 +991,18 @@ shampoo_status shampoo_set_root_options(shampoo_ctx* ctx, double tol, int max_it
   return SHAMPOO_OK;
 }
 
+shampoo_status shampoo_set_root_method(shampoo_ctx* ctx, int method, int slices) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (method != SHAMPOO_ROOTS_FP64 && method != SHAMPOO_ROOTS_INT8_EMULATED)
+    return fail(ctx, SHAMPOO_EINVAL, "unknown root method");
+  if (method == SHAMPOO_ROOTS_INT8_EMULATED && (slices < 4 || slices > kOzMaxSlices))
+    return fail(ctx, SHAMPOO_EINVAL, "slices must be in [4, 7]");
+  if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "an asynchronous root job is in flight");
+  ctx->root_method = method;
+  if (method == SHAMPOO_ROOTS_INT8_EMULATED) ctx->oz_slices = slices;
+  return SHAMPOO_OK;
+}
+
 int shampoo_num_matrices(const shampoo_ctx* ctx) { return ctx ? ctx->nmat : 0; }
 
 shampoo_status shampoo_matrix_info(const shampoo_ctx* ctx, int index, int* size, int* root_p) {
@@ -982,11 +1065,22 @@ shampoo_status shampoo_profile_entry(shampoo_ctx* ctx, int index, char* name, in
 shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch, int n, int p,
                                             float eps, double tol, int max_iters, int32_t* iters,
                                             void* stream) {
+  return shampoo_batched_inverse_root_ex(A, X, batch, n, p, eps, tol, max_iters, iters, stream,
+                                         SHAMPOO_ROOTS_FP64, 0);
+}
+
+shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int batch, int n, int p,
+                                               float eps, double tol, int max_iters, int32_t* iters,
+                                               void* stream, int method, int slices) {
   if (!A || !X || batch < 1 || n < 1 || n > 1024 || (p != 2 && p != 4) || !(eps > 0.f) ||
-      !(tol > 0.0) || max_iters < 1 || max_iters > 1000)
+      !(tol > 0.0) || max_iters < 1 || max_iters > 1000 ||
+      (method != SHAMPOO_ROOTS_FP64 && method != SHAMPOO_ROOTS_INT8_EMULATED) ||
+      (method == SHAMPOO_ROOTS_INT8_EMULATED && (slices < 4 || slices > kOzMaxSlices)))
     return fail(nullptr, SHAMPOO_EINVAL, "bad argument to shampoo_batched_inverse_root");
   shampoo_ctx tmp;   // carries the allocations and the error text only
   shampoo_ctx* ctx = &tmp;
+  const bool use_oz = method == SHAMPOO_ROOTS_INT8_EMULATED;
+  int kerr = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int S = (n + kTile - 1) / kTile * kTile;
   const size_t per = 7 * (size_t)S * S * sizeof(double);
@@ -1010,12 +1104,31 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
   }
   if ((e = cudaMallocHost(&ctx->h_count, 2 * sizeof(int))) != cudaSuccess ||
       (e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming)) != cudaSuccess ||
-      (e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming)) != cudaSuccess) {
+      (e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming)) != cudaSuccess ||
+      (e = dalloc(ctx, &ctx->d_err, 1)) != cudaSuccess ||
+      (e = cudaMemsetAsync(ctx->d_err, 0, sizeof(int), st)) != cudaSuccess) {
     res = cuda_fail(ctx, e, "set-up");
     goto done;
   }
+  if (use_oz) {
+    ctx->S = S;
+    ctx->newton_chunk = chunk;
+    if ((res = ensure_ozaki(ctx)) != SHAMPOO_OK) goto done;
+    w.q = ctx->nw.q;
+    w.qe = ctx->nw.qe;
+    w.qcap = ctx->nw.qcap;
+    w.qs = slices;
+  }
   res = run_newton(ctx, nullptr, hm, dm, dr, A, (int64_t)n * n, n, 0, X, (int64_t)n * n, n, S, eps, tol,
-                   max_iters, chunk, w, nullptr, iters, ctx->h_count, ctx->ev, st, &nf, &mi, nullptr);
+                   max_iters, chunk, w, nullptr, iters, ctx->h_count, ctx->ev, st, &nf, &mi, nullptr,
+                   use_oz ? &ctx->oz : nullptr, ctx->d_err);
+  if (res == SHAMPOO_OK && use_oz) {
+    if ((e = cudaMemcpyAsync(&kerr, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
+      res = cuda_fail(ctx, e, "error word");
+    else if (kerr)
+      res = fail(ctx, SHAMPOO_ECUDA, "a tensor-core kernel timed out waiting on its pipeline");
+  }
   if (res == SHAMPOO_OK && nf) res = fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
 done:
   cudaStreamSynchronize(st);

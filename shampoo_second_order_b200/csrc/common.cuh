@@ -16,6 +16,11 @@ __device__ __forceinline__ float grad_at(const void* p, int64_t i, int bf16) {
   return __ldg(reinterpret_cast<const float*>(p) + i);
 }
 
+// Scaling s_k of Newton step k of matrix m (1 past the scaled steps).
+__device__ __forceinline__ double newton_sched(const NewtonWork& w, int m, int k) {
+  return k < w.nsched[m] ? w.sched[(size_t)m * kSched + k] : 1.0;
+}
+
 // Warp sum / max.
 __device__ __forceinline__ double warp_sum(double v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

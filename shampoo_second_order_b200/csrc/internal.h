@@ -101,6 +101,23 @@ struct NewtonWork {
   int* state;                   // [nmat] 0 running, 1 converged, 2 failed, 3 diverged,
                                 //        4 one X-only step left
   int* count;                   // [1] matrices still active after a check
+  // int8 slices of the iterates for the emulated-float64 products (k_ozaki.cu):
+  //   q   int8 [kOzSets][qs][qcap][S][S], slice k of set z for matrix m at
+  //       plane (z * qs + k) * qcap + m
+  //   qe  int32 [kOzSets][qcap][S], the row exponents
+  int8_t* q;
+  int* qe;
+  int qs;                       // slices per value
+  int qcap;                     // matrices the slice planes hold
+};
+
+// Matrix sets sliced for the emulated products.
+enum : int { kOzX = 0, kOzT = 1, kOzT2 = 2, kOzT4 = 3, kOzM = 4, kOzSets = 5 };
+constexpr int kOzMaxSlices = 7;   // 7 accumulators of 64 TMEM columns
+// TMA descriptors over the int8 slice planes [kOzSets * qs * qcap][S][S]
+// (128-byte swizzle, K-major): a  box 128 x 128 (row tile), b  box 128 x 64.
+struct OzakiMaps {
+  CUtensorMap a, b;
 };
 // Set up X0, M0, T0 for `nm` matrices read from `A` (float32, slot-strided
 // `a_stride` elements apart, row stride `lda`, valid side mats[i].size).
@@ -122,6 +139,17 @@ void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWo
 void launch_newton_step_b(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
 void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);
 void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s);
+
+// ---------------- emulated float64 Newton products (k_ozaki.cu) ----------------
+// Slice the listed sets (bit z of `sets` = set z) of every running matrix:
+// per row an exponent e with max|v| < 2^e and qs signed 7-bit slices of the
+// truncated fixed-point value v 2^-e.
+cudaError_t launch_ozaki_split(const NewtonMat* mats, int nm, int S, int it, unsigned sets, NewtonWork w,
+                               cudaStream_t s);
+// The products of one Newton step on the int8 tensor cores; step = 0 (A:
+// X T and T T), 1 (B: T2 T2, p = 4), 2 (C: T^p M with the residual and next T).
+cudaError_t launch_ozaki_step(const OzakiMaps& maps, int step, const NewtonMat* mats, int nm, int S, int it,
+                              NewtonWork w, int* err, cudaStream_t s);
 // Write the roots back as float32.  keep_old: leave a failed matrix's slot
 // untouched if has_root[slot] is set; else write c^{-1} I.
 // A diverged matrix is skipped unless final_pass (it will be retried).

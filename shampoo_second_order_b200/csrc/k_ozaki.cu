@@ -1,0 +1,449 @@
+// Float64-accurate products of the Newton iteration on the int8 tensor
+// cores: the Ozaki scheme (Ozaki, Ogita, Oishi, Rump 2012) in its integer
+// form (Ootomo, Ozaki, Yokota 2024), for the coupled Newton iteration of
+// k_roots.cu (podcast transcript, segment 12: the roots need double
+// precision).  tcgen05 has no float64 kind; its int8 kind multiplies exactly.
+//
+// Each row r of an iterate Z is written as
+//   Z[r][:] ~ 2^{e_r} sum_{k=1..qs} q_k[r][:] 2^{-7k},   q_k in [-127, 127],
+// the qs 7-bit digits of the fixed-point value |Z[r][:]| 2^{-e_r}, truncated
+// toward zero and signed like Z, with e_r the smallest exponent such that
+// max|Z[r][:]| < 2^{e_r}.  A product C = A B of two such iterates (B is
+// symmetric: every iterate is a polynomial in the statistic, so B's columns
+// are its rows) becomes
+//   C[i][j] ~ 2^{e_i + f_j} sum_{a + b <= qs + 1} 2^{-7(a+b)} (q^A_a (q^B_b)^T)[i][j],
+// where each q_a q_b^T is an exact int8 x int8 -> int32 product on the
+// tensor cores (|entry| <= S 127^2 < 2^24 for S <= 1024).  Pairs with the
+// same a + b share one int32 accumulator (at most qs pairs, still exact), so
+// a tile keeps qs accumulators in TMEM and turns them into float64 once.
+// Truncating each value and dropping the pairs with a + b > qs + 1 leaves an
+// error of order S 2^{-7 qs} 2^{e_i + f_j} per entry: 2^-42 S relative to the
+// row and column scales for the default qs = 6, against 2^-53 per rounding
+// of a float64 product.
+//
+// Kernels:
+//   ozaki_split  per row: exponent and qs int8 slice planes of a float64 iterate
+//   ozaki_gemm   persistent, warp-specialised: lane 0 of warp 0 loads the
+//                slice planes by TMA (a stage = one slice of A's 128-row
+//                tile and of B's 64-row tile over 128 K), lane 0 of warp 1
+//                issues the int8 MMAs of every pair as soon as its slices
+//                are in, warps 2-5 combine the accumulators in float64, scale
+//                them and run the step's epilogue.
+// Output tiles are 128 x 64 over the upper triangle; every entry with
+// r <= c is written by its tile and mirrored to (c, r), as in k_roots.cu.
+#include <float.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace shampoo {
+
+namespace {
+
+enum : int { kRunning = 0, kFinal = 4 };    // NewtonWork.state values read here
+constexpr int kBadExp = 1 << 20;             // exponent of a row holding NaN or Inf
+constexpr int kTileM = 128, kTileN = 64, kKBytes = 128;
+constexpr int kABytes = kTileM * kKBytes;    // 16 KB: one slice of the row tile
+constexpr int kBBytes = kTileN * kKBytes;    // 8 KB: one slice of the column tile
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kStages = 9;                   // one K chunk of 7 slices plus look-ahead
+constexpr uint32_t kIdesc = tc::idesc_s8(kTileM, kTileN);
+
+// ---------------------------------------------------------------------------
+// split
+// ---------------------------------------------------------------------------
+struct SplitJobs {
+  const double* src[2];   // float64 [qcap][S][S]
+  int set[2];
+};
+
+// grid: x = group of 8 rows, y = matrix, z = job.  One warp per row; lane l
+// holds the columns 128 i + 4 l .. + 3.
+__global__ void __launch_bounds__(256) ozaki_split_kernel(const NewtonMat* __restrict__ mats, int S,
+                                                          SplitJobs jobs, NewtonWork w) {
+  const int m = blockIdx.y;
+  if (w.state[m] != kRunning) return;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= S) return;
+  const int set = jobs.set[blockIdx.z];
+  const double* row = jobs.src[blockIdx.z] + (size_t)m * S * S + (size_t)r * S;
+  const int qs = w.qs;
+  double v[32];
+  double mx = 0.0;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = 128 * i + 4 * lane;
+    if (c < S) {
+      const double2 a = *reinterpret_cast<const double2*>(row + c);
+      const double2 b = *reinterpret_cast<const double2*>(row + c + 2);
+      v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = b.x; v[4 * i + 3] = b.y;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bad |= !(fabs(v[4 * i + j]) <= DBL_MAX);
+        mx = fmax(mx, fabs(v[4 * i + j]));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * i + j] = 0.0;
+    }
+  }
+  mx = warp_max(mx);
+  bad = __any_sync(0xffffffffu, bad);
+  int e = 0;
+  if (!bad && mx > 0.0) frexp(mx, &e);        // mx = f 2^e, f in [0.5, 1): every |v| < 2^e
+  // a row far below the float64 range of its neighbours counts as zero
+  const bool zero = bad || mx == 0.0 || e < -900;
+  const double scale = zero ? 0.0 : ldexp(1.0, 7 * qs - e);
+  int8_t* q0 = w.q + ((size_t)set * qs * w.qcap + m) * S * S + (size_t)r * S;
+  const size_t plane = (size_t)w.qcap * S * S;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = 128 * i + 4 * lane;
+    if (c >= S) continue;
+    unsigned long long f[4];
+    bool neg[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[j] = (unsigned long long)(fabs(v[4 * i + j]) * scale);   // < 2^{7 qs}: exact scaling, truncated
+      neg[j] = v[4 * i + j] < 0.0;
+    }
+    for (int k = 0; k < qs; ++k) {
+      const int sh = 7 * (qs - 1 - k);
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int d = (int)((f[j] >> sh) & 127ull);
+        if (neg[j]) d = -d;
+        word |= (uint32_t)(uint8_t)(int8_t)d << (8 * j);
+      }
+      *reinterpret_cast<uint32_t*>(q0 + k * plane + c) = word;
+    }
+  }
+  if (lane == 0) w.qe[((size_t)set * w.qcap + m) * S + r] = bad ? kBadExp : (zero ? 0 : e);
+}
+
+// ---------------------------------------------------------------------------
+// products
+// ---------------------------------------------------------------------------
+struct OzArgs {
+  const NewtonMat* mats;
+  NewtonWork w;
+  int S, it, step, ntri;
+  int* err;
+};
+
+// Tile idx of a matrix's upper triangle, row-major: row tile ti covers rows
+// 128 ti .., column tile tj columns 64 tj ..; tj runs from 2 ti.
+__host__ __device__ inline void oz_tile(int idx, int S, int& ti, int& tj) {
+  const int tc = S / kTileN;
+  ti = 0;
+  while (idx >= tc - 2 * ti) {
+    idx -= tc - 2 * ti;
+    ++ti;
+  }
+  tj = 2 * ti + idx;
+}
+
+int oz_ntri(int S) {
+  const int tc = S / kTileN, tr = (S + kTileM - 1) / kTileM;
+  int n = 0;
+  for (int ti = 0; ti < tr; ++ti) n += tc - 2 * ti > 0 ? tc - 2 * ti : 0;
+  return n;
+}
+
+struct OzTile {
+  int m, job, i0, j0, setA, setB;
+  bool skip;
+};
+
+__device__ __forceinline__ OzTile oz_decode(int t, const OzArgs& a) {
+  const int njobs = a.step == 0 ? 2 : 1;
+  OzTile x{};
+  x.m = t / (njobs * a.ntri);
+  const int r = t % (njobs * a.ntri);
+  x.job = r / a.ntri;
+  int ti, tj;
+  oz_tile(r % a.ntri, a.S, ti, tj);
+  x.i0 = ti * kTileM;
+  x.j0 = tj * kTileN;
+  const int st = a.w.state[x.m];
+  const int p = a.mats[x.m].p;
+  if (a.step == 0) {
+    x.skip = x.job == 0 ? !(st == kRunning || st == kFinal) : st != kRunning;
+    x.setA = x.job == 0 ? kOzX : kOzT;
+    x.setB = kOzT;
+  } else if (a.step == 1) {
+    x.skip = st != kRunning || p != 4;
+    x.setA = x.setB = kOzT2;
+  } else {
+    x.skip = st != kRunning;
+    x.setA = p == 4 ? kOzT4 : kOzT2;
+    x.setB = kOzM;
+  }
+  return x;
+}
+
+__global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                                                            const __grid_constant__ CUtensorMap map_b,
+                                                            OzArgs args, int ntiles) {
+  extern __shared__ uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = args.S, qs = args.w.qs, qcap = args.w.qcap;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;    // accumulators ready for the epilogue
+  uint64_t* tempty = tfull + 1;         // accumulators read out by the epilogue
+  uint64_t* drain = tempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(tfull, 1);
+    tc::mbar_init(tempty, 128);
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 512);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = (S + kKBytes - 1) / kKBytes;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    int g = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      const OzTile x = oz_decode(t, args);
+      if (x.skip) continue;
+      bool ok = true;
+      for (int kc = 0; kc < nk && ok; ++kc)
+        for (int k = 0; k < qs; ++k, ++g) {
+          const int s = g % kStages;
+          if (g >= kStages && !tc::mbar_wait(&empty[s], ((g / kStages) - 1) & 1)) {
+            *abort_flag = 1;
+            atomicExch(args.err, tc::kErrTimeout);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          tc::mbar_expect_tx(&full[s], kStageBytes);
+          tc::tma_load_3d(st, &map_a, &full[s], kc * kKBytes, x.i0, (x.setA * qs + k) * qcap + x.m);
+          tc::tma_load_3d(st + kABytes, &map_b, &full[s], kc * kKBytes, x.j0, (x.setB * qs + k) * qcap + x.m);
+        }
+      if (!ok) break;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    int g = 0, i = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      const OzTile x = oz_decode(t, args);
+      if (x.skip) continue;
+      if (i >= 1 && !tc::mbar_wait(tempty, (i - 1) & 1)) {
+        *abort_flag = 1;
+        atomicExch(args.err, tc::kErrTimeout);
+        break;
+      }
+      tc::fence_after_sync();
+      uint32_t inited = 0;   // accumulators written in this tile
+      bool ok = true;
+      const uint32_t ring = tc::smem_u32(smem);
+      for (int kc = 0; kc < nk && ok; ++kc) {
+        const int g0 = g;   // ring position of this chunk's slice 0
+        for (int k = 0; k < qs; ++k, ++g) {
+          const int s = g % kStages;
+          if (!tc::mbar_wait(&full[s], (g / kStages) & 1)) {
+            *abort_flag = 1;
+            atomicExch(args.err, tc::kErrTimeout);
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          // every pair (a, b), a + b <= qs - 1 (0-based), whose later slice is k
+          for (int o = 0; o <= k && o + k <= qs - 1; ++o) {
+            for (int sw = 0; sw < (o < k ? 2 : 1); ++sw) {   // (k, o), then (o, k) for o < k
+              const int ia = sw ? o : k, ib = sw ? k : o;
+              const int d = ia + ib;
+              const uint32_t dt = tmem + d * kTileN;
+              const uint32_t sa = ring + ((g0 + ia) % kStages) * kStageBytes;
+              const uint32_t sb = ring + ((g0 + ib) % kStages) * kStageBytes + kABytes;
+#pragma unroll
+              for (int kk = 0; kk < kKBytes / 32; ++kk) {
+                const uint64_t da = tc::smem_desc(sa + kk * 32, 16, 1024);
+                const uint64_t db = tc::smem_desc(sb + kk * 32, 16, 1024);
+                tc::mma_i8(dt, da, db, kIdesc, ((inited >> d) & 1u) | (kk > 0));
+              }
+              inited |= 1u << d;
+            }
+          }
+        }
+        if (!ok) break;
+        // this chunk's stages are free once its MMAs have read them
+        for (int k = 0; k < qs; ++k) tc::mma_commit(&empty[(g - qs + k) % kStages]);
+      }
+      if (!ok) break;
+      tc::mma_commit(tfull);
+      ++i;
+    }
+    tc::mma_commit(drain);
+    tc::mbar_wait(drain, 0);
+  } else if (warp >= 2) {
+    // ---------------- epilogue ----------------
+    const int q = warp & 3;
+    int i = 0;
+    const NewtonWork& w = args.w;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const OzTile x = oz_decode(t, args);
+      if (x.skip) continue;
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tfull, i & 1) && !*abort_flag);
+      if (!ok) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          atomicExch(args.err, tc::kErrTimeout);
+        }
+        break;
+      }
+      tc::fence_after_sync();
+      const int m = x.m, rl = q * 32 + lane, r = x.i0 + rl;
+      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+      double acc[2][32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[c][j] = 0.0;
+        for (int d = 0; d < qs; ++d) {
+          float v[32];
+          tc::tmem_ld32(trow + d * kTileN + c * 32, v);
+          const double wd = ldexp(1.0, -7 * (d + 2));
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[c][j] = fma((double)__float_as_int(v[j]), wd, acc[c][j]);
+        }
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(tempty);   // the next tile's MMAs may overwrite the accumulators
+      ++i;
+
+      const size_t base = (size_t)m * S * S;
+      const int ea = r < S ? w.qe[((size_t)x.setA * qcap + m) * S + r] : 0;
+      const int* eb = w.qe + ((size_t)x.setB * qcap + m) * S;
+      const int p = args.mats[m].p;
+      double mul = 1.0;
+      double* C;
+      if (args.step == 0 && x.job == 0) {            // X_next = s_k^{1/p} X T
+        const double sk = newton_sched(w, m, args.it);
+        if (sk != 1.0) mul = pow(sk, 1.0 / p);
+        C = w.X[(args.it + 1) & 1] + base;
+      } else if (args.step == 0) {
+        C = w.T2 + base;                             // T2 = T T
+      } else if (args.step == 1) {
+        C = w.T4 + base;                             // T4 = T2 T2
+      } else {
+        mul = newton_sched(w, m, args.it);           // M_next = s_k T^p M
+        C = w.M[(args.it + 1) & 1] + base;
+      }
+      const bool resid = args.step == 2;
+      const double sn = resid ? newton_sched(w, m, args.it + 1) : 0.0, pinv = 1.0 / p;
+      const int n = args.mats[m].size;
+      double dev = 0.0, f2 = 0.0;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int col = x.j0 + c * 32 + j;
+          if (r >= S || col >= S || r > col) continue;
+          const int e2 = eb[col];
+          const double v = (ea == kBadExp || e2 == kBadExp) ? __longlong_as_double(0x7ff8000000000000ll)
+                                                          : ldexp(acc[c][j], ea + e2) * mul;
+          C[(size_t)r * S + col] = v;
+          if (r < col) C[(size_t)col * S + r] = v;
+          if (resid) {
+            const double dl = (r == col) ? 1.0 : 0.0;
+            if (r < n && col < n) {
+              double xd = fabs(v - dl);
+              if (!(xd <= DBL_MAX)) xd = INFINITY;
+              dev = fmax(dev, xd);
+              f2 += (r == col ? 1.0 : 2.0) * xd * xd;   // an entry above the diagonal counts for its mirror too
+            }
+            const double tn = ((p + 1) * dl - sn * v) * pinv;   // next T = ((p+1) I - s_{k+1} M_next) / p
+            w.T[base + (size_t)r * S + col] = tn;
+            if (r < col) w.T[base + (size_t)col * S + r] = tn;
+          }
+        }
+      }
+      if (resid) {
+        dev = warp_max(dev);
+        f2 = warp_sum(f2);
+        if (lane == 0) {
+          atomicMax(&w.resid[m], static_cast<unsigned long long>(__double_as_longlong(dev)));
+          atomicAdd(&w.fro2[m], f2);
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+int sm_count_oz() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_ozaki_split(const NewtonMat* mats, int nm, int S, int it, unsigned sets, NewtonWork w,
+                               cudaStream_t s) {
+  // the float64 source of each set at step `it` (X and M: the buffers step it wrote)
+  const double* src[kOzSets] = {w.X[it & 1], w.T, w.T2, w.T4, w.M[it & 1]};
+  SplitJobs jobs{};
+  int nj = 0;
+  for (int z = 0; z < kOzSets; ++z) {
+    if (!(sets >> z & 1u)) continue;
+    if (nj == 2) {
+      ozaki_split_kernel<<<dim3((S + 7) / 8, nm, nj), 256, 0, s>>>(mats, S, jobs, w);
+      nj = 0;
+    }
+    jobs.src[nj] = src[z];
+    jobs.set[nj] = z;
+    ++nj;
+  }
+  if (nj) ozaki_split_kernel<<<dim3((S + 7) / 8, nm, nj), 256, 0, s>>>(mats, S, jobs, w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ozaki_step(const OzakiMaps& maps, int step, const NewtonMat* mats, int nm, int S, int it,
+                              NewtonWork w, int* err, cudaStream_t s) {
+  static bool configured = false;
+  const int smem = kStages * kStageBytes + 1024 + 256;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(ozaki_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  OzArgs a{};
+  a.mats = mats; a.w = w; a.S = S; a.it = it; a.step = step; a.ntri = oz_ntri(S); a.err = err;
+  const int ntiles = nm * (step == 0 ? 2 : 1) * a.ntri;
+  const int grid = ntiles < sm_count_oz() ? ntiles : sm_count_oz();
+  ozaki_gemm_kernel<<<grid, 192, smem, s>>>(maps.a, maps.b, a, ntiles);
+  return cudaGetLastError();
+}
+
+}  // namespace shampoo

@@ -236,7 +236,9 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
     double v;
     const bool valid = r < mt.size && c < mt.size;
     if (valid) {
-      v = (double)sym_at(a, lda, upper, r, c);
+      // a full input is read through its symmetric part (exact when symmetric)
+      v = upper ? (double)sym_at(a, lda, upper, r, c)
+                : 0.5 * ((double)a[(size_t)r * lda + c] + (double)a[(size_t)c * lda + r]);
       if (r == c) v += rd;
       v *= inv_cp;
     } else {
@@ -406,9 +408,7 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
   w.nsched[m] = ns;
 }
 
-__device__ __forceinline__ double sched_at(const NewtonWork& w, int m, int k) {
-  return k < w.nsched[m] ? w.sched[(size_t)m * kSched + k] : 1.0;
-}
+__device__ __forceinline__ double sched_at(const NewtonWork& w, int m, int k) { return newton_sched(w, m, k); }
 
 // T0 = ((p+1) I - s_0 M0) / p.  grid: x = row, y = matrix.
 __global__ void __launch_bounds__(256) newton_t0_kernel(const NewtonMat* __restrict__ mats, int S,

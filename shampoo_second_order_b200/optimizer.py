@@ -77,6 +77,11 @@ class Shampoo:
     def set_root_options(self, tol, max_iters):
         L.shampoo_set_root_options(self.ctx, tol, max_iters)
 
+    def set_root_method(self, method="fp64", slices=6):
+        """method "fp64" (float64 Newton products) or "int8" (the same products
+        emulated on the int8 tensor cores with `slices` 7-bit slices)."""
+        L.shampoo_set_root_method(self.ctx, _METHODS[method], slices)
+
     def root_iterations(self):
         return L.shampoo_root_iterations(self.ctx)
 
@@ -113,8 +118,10 @@ class Shampoo:
             pass
 
 
-def batched_inverse_root(A, p, eps, tol=1e-6, max_iters=100, stream=None):
+def batched_inverse_root(A, p, eps, tol=1e-6, max_iters=100, stream=None, method="fp64", slices=6):
     """X = (A + eps I)^{-1/p} for a float32 CUDA tensor A [batch, n, n].
+    method: "fp64" (float64 products) or "int8" (float64 products emulated
+    on the int8 tensor cores with `slices` 7-bit slices).
     Returns (X, iters) with iters an int32 CUDA tensor (negative = gave up)."""
     import torch
     assert A.is_cuda and A.dtype == torch.float32 and A.dim() == 3 and A.is_contiguous()
@@ -123,6 +130,9 @@ def batched_inverse_root(A, p, eps, tol=1e-6, max_iters=100, stream=None):
     iters = torch.empty(batch, dtype=torch.int32, device=A.device)
     if stream is None:
         stream = torch.cuda.current_stream()
-    L.shampoo_batched_inverse_root(A.data_ptr(), X.data_ptr(), batch, n, p, eps, tol, max_iters,
-                                   iters.data_ptr(), stream.cuda_stream)
+    L.shampoo_batched_inverse_root_ex(A.data_ptr(), X.data_ptr(), batch, n, p, eps, tol, max_iters,
+                                      iters.data_ptr(), stream.cuda_stream, _METHODS[method], slices)
     return X, iters
+
+
+_METHODS = {"fp64": L.ROOTS_FP64, "int8": L.ROOTS_INT8_EMULATED}

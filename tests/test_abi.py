@@ -84,6 +84,7 @@ def test_null_context_calls(lib):
     assert lib.shampoo_compute_roots_async(None) == L.EINVAL
     assert lib.shampoo_install_roots(None, 0, None) == L.EINVAL
     assert lib.shampoo_roots_generation(None) == -1
+    assert lib.shampoo_set_root_method(None, 1, 6) == L.EINVAL
     lib.shampoo_destroy(None)
 
 
@@ -99,6 +100,13 @@ def test_batched_root_rejects_bad_arguments(lib, args):
     a, x, batch, n, p, eps, tol, mi = args
     st = lib.shampoo_batched_inverse_root(C.c_void_p(a), C.c_void_p(x), batch, n, p, eps, tol, mi,
                                           None, None)
+    assert st == L.EINVAL
+
+
+@pytest.mark.parametrize("method,slices", [(2, 6), (1, 3), (1, 8), (-1, 6)])
+def test_batched_root_ex_rejects_bad_method(lib, method, slices):
+    st = lib.shampoo_batched_inverse_root_ex(C.c_void_p(8), C.c_void_p(8), 1, 64, 4, 1e-6, 1e-6, 100,
+                                             None, None, method, slices)
     assert st == L.EINVAL
 
 

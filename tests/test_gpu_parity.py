@@ -55,10 +55,11 @@ def pieces(shape, b):
 
 
 def run_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, interval, seed, gstd,
-             check_every=True, check_state=True):
+             check_every=True, check_state=True, method="fp64"):
     from shampoo_second_order_b200 import Shampoo
     o = ShampooOracle(shapes, b, beta2, eps, 4, graft, mu)
     opt = Shampoo(shapes, b, beta2, eps, 4, graft, mu, gdtype)
+    opt.set_root_method(method)
     W0 = wl.make_params(shapes, seed)
     Wo = [w.astype(np.float64) for w in W0]
     Wd = [torch.from_numpy(w).cuda() for w in W0]
@@ -172,6 +173,71 @@ def test_batched_root_kappa_sweep_full_size():
             if kappa[i] <= 1e6:
                 assert iters[i] > 0
                 assert rel(X[i], ref) <= ROOT_TOL, (p, i, kappa[i], rel(X[i], ref))
+
+
+@pytest.mark.parametrize("n", [64, 100, 192, 512])
+@pytest.mark.parametrize("p", [2, 4])
+def test_batched_root_int8_emulated_vs_oracle(n, p):
+    """Newton with its products emulated on the int8 tensor cores (6 slices)
+    reaches the oracle's root like the float64 products do, in the same
+    number of steps give or take one."""
+    from shampoo_second_order_b200 import batched_inverse_root
+    A, _ = wl.spd_batch(6, n, seed=n + p, log10_kappa=(2.0, 6.0))
+    dA = torch.from_numpy(A.astype(np.float32)).cuda()
+    X, iters = batched_inverse_root(dA, p, 1e-6, method="int8")
+    _, iters64 = batched_inverse_root(dA, p, 1e-6)
+    X = X.cpu().numpy()
+    iters, iters64 = iters.cpu().numpy(), iters64.cpu().numpy()
+    assert (iters > 0).all() and (np.abs(iters - iters64) <= 1).all(), (iters, iters64)
+    for i in range(6):
+        ref = inverse_root(A[i].astype(np.float32).astype(np.float64), 1e-6, p)
+        assert rel(X[i], ref) <= ROOT_TOL, (i, rel(X[i], ref))
+
+
+def test_batched_root_int8_emulated_kappa_sweep():
+    """The 256 x 512 kappa sweep (1e2..1e8) through the emulated products,
+    sampled; every matrix with kappa <= 1e6 within 1e-3 of the oracle."""
+    from shampoo_second_order_b200 import batched_inverse_root
+    c = wl.ROOTS_CONFIG
+    A, lam = wl.spd_batch(c["batch"], c["n"], c["seed"], c["log10_kappa"])
+    A32 = A.astype(np.float32)
+    dA = torch.from_numpy(A32).cuda()
+    kappa = lam.max(1) / lam.min(1)
+    for p in c["ps"]:
+        X, iters = batched_inverse_root(dA, p, c["eps"], c["tol"], method="int8")
+        X = X.cpu().numpy()
+        iters = iters.cpu().numpy()
+        for i in list(range(0, c["batch"], 16)) + [c["batch"] - 1]:
+            if kappa[i] <= 1e6:
+                ref = inverse_root(A32[i].astype(np.float64), c["eps"], p)
+                assert iters[i] > 0
+                assert rel(X[i], ref) <= ROOT_TOL, (p, i, kappa[i], rel(X[i], ref))
+
+
+def test_batched_root_int8_nan_input_fails_that_matrix_only():
+    from shampoo_second_order_b200 import batched_inverse_root
+    A = np.stack([np.eye(128, dtype=np.float32) * 2, np.eye(128, dtype=np.float32)])
+    A[1, 3, 3] = np.nan
+    X, iters = batched_inverse_root(torch.from_numpy(A).cuda(), 4, 1e-6, method="int8")
+    iters = iters.cpu().numpy()
+    assert iters[0] >= 0 and iters[1] < 0
+    assert np.allclose(X[0].cpu().numpy(), (2 + 1e-6) ** -0.25 * np.eye(128), rtol=1e-6)
+
+
+@pytest.mark.parametrize("gdtype", ["f32", "bf16"])
+def test_ragged_mixed_set_int8_emulated_roots(gdtype):
+    shapes = [(200, 130), (64, 64), (19, 200), (130,), (64,), (1, 77)]
+    w = run_pair(shapes, 64, 0.99, 1e-6, 1, 0.9, 0.1, gdtype, steps=6, interval=3, seed=7,
+                 gstd=1e-2, method="int8")
+    assert_worst(w)
+
+
+def test_transformer_layer_b512_int8_emulated_roots():
+    c = wl.CONFIGS["transformer_layer_b512"]
+    w = run_pair(c["shapes"], c["block_size"], c["beta2"], c["eps"], c["graft"], c["momentum"],
+                 c["lr"], c["grad_dtype"], 21, c["root_interval"], c["seed"], c["grad_std"],
+                 check_every=False, method="int8")
+    assert_worst(w)
 
 
 # --------------------------------------------------------------------------
@@ -330,7 +396,8 @@ def test_resnet50_full_set():
 # asynchronous roots (podcast transcript, segment 16): the steps keep using
 # the roots in place while the next ones are computed, then swap them in
 # --------------------------------------------------------------------------
-def run_async_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, submit, wait_at, seed, gstd):
+def run_async_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, submit, wait_at, seed, gstd,
+                   method="fp64"):
     """Roots synchronously at step 0; an asynchronous job queued after the
     statistics of each step in `submit`; a blocking install before the apply
     of each step in `wait_at`.  The library swaps a finished job in at an
@@ -341,6 +408,7 @@ def run_async_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, submit, 
     from shampoo_second_order_b200 import Shampoo
     o = ShampooOracle(shapes, b, beta2, eps, 4, graft, mu)
     opt = Shampoo(shapes, b, beta2, eps, 4, graft, mu, gdtype)
+    opt.set_root_method(method)
     W0 = wl.make_params(shapes, seed)
     Wo = [w.astype(np.float64) for w in W0]
     Wd = [torch.from_numpy(w).cuda() for w in W0]
@@ -382,11 +450,11 @@ def run_async_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, submit, 
     return worst, installs
 
 
-@pytest.mark.parametrize("gdtype", ["f32", "bf16"])
-def test_async_roots_ragged_set(gdtype):
+@pytest.mark.parametrize("gdtype,method", [("f32", "fp64"), ("bf16", "fp64"), ("f32", "int8")])
+def test_async_roots_ragged_set(gdtype, method):
     shapes = [(200, 130), (64, 64), (19, 200), (130,), (64,), (1, 77)]
     w, installs = run_async_pair(shapes, 64, 0.99, 1e-6, 1, 0.0, 0.1, gdtype, steps=9,
-                                 submit=(2, 5), wait_at=(4, 8), seed=7, gstd=1e-2)
+                                 submit=(2, 5), wait_at=(4, 8), seed=7, gstd=1e-2, method=method)
     assert w["dW"] <= STEP_TOL and w["W"] <= STEP_TOL, w
     assert len(installs) == 2 and 2 <= installs[0] <= 4 and 5 <= installs[1] <= 8, installs
 
