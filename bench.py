@@ -284,6 +284,14 @@ def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak, slices
                     "MEASURED_PEAKS.json bf16_tflops (burst)")
         else:
             work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / launches, "MEASURED_PEAKS.json hbm_gbs")
+    elif top == "ozaki_split":
+        S = -(-cfg["block_size"] // 64) * 64
+        sets = 0
+        for (n, prods), k in zip(matrix_sizes(cfg), iters_sum):
+            k = k if k >= 0 else -1 - k
+            sets += 3 * n_root_steps + k * (5 if prods == 4 else 4)   # X T M at the start; X T2 (T4) M T per step
+        by = sets * S * S * (8 + slices)                              # read float64, write the slices
+        work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")
     elif top == "newton_lanczos":
         by = sum(12 * 8 * n * n for n, _ in matrix_sizes(cfg)) * n_root_steps
         work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")

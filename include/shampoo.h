@@ -223,8 +223,8 @@ shampoo_status shampoo_set_root_options(shampoo_ctx* ctx, double tol, int max_it
  *          cores.  Per entry the error is of order n 2^{-7 slices} times the
  *          row and column scales (2^-42 n for 6 slices), against 2^-53 for a
  *          float64 product.
- *  slices  4..7 for the emulated method (6 recommended); ignored otherwise.
- * The emulated method allocates 35 int8 planes of b x b bytes (5 iterates x 7
+ *  slices  4..6 for the emulated method (6 recommended); ignored otherwise.
+ * The emulated method allocates 30 int8 planes of b x b bytes (5 iterates x 6
  * slices) per matrix of a Newton chunk on first use.  SHAMPOO_EBUSY while an
  * asynchronous root job runs.
  */
@@ -313,7 +313,7 @@ shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
 /*
  * shampoo_batched_inverse_root_ex -- shampoo_batched_inverse_root with the
  * product method of shampoo_set_root_method (method, slices).  The emulated
- * method also allocates its int8 slice planes (35 n' x n' bytes per matrix in
+ * method also allocates its int8 slice planes (30 n' x n' bytes per matrix in
  * flight, n' = n rounded up to 64) and frees them before returning.
  */
 shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int batch,

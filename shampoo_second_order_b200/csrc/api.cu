@@ -461,14 +461,14 @@ shampoo_status ensure_ozaki(shampoo_ctx* ctx) {
   auto fn = encode_fn();
   cuuint64_t dims[3] = {(cuuint64_t)S, (cuuint64_t)S, (cuuint64_t)planes};
   cuuint64_t strides[2] = {(cuuint64_t)S, (cuuint64_t)S * S};
-  cuuint32_t box_a[3] = {128, 128, 1}, box_b[3] = {128, 64, 1};
+  cuuint32_t box_a[3] = {64, 128, 1}, box_b[3] = {64, 64, 1};
   cuuint32_t es[3] = {1, 1, 1};
   if (!fn ||
       fn(&ctx->oz.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box_a, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
       fn(&ctx->oz.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box_b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return fail(ctx, SHAMPOO_ECUDA, "cuTensorMapEncodeTiled failed for the slice planes");
   ctx->nw.q = q;
@@ -996,7 +996,7 @@ shampoo_status shampoo_set_root_method(shampoo_ctx* ctx, int method, int slices)
   if (method != SHAMPOO_ROOTS_FP64 && method != SHAMPOO_ROOTS_INT8_EMULATED)
     return fail(ctx, SHAMPOO_EINVAL, "unknown root method");
   if (method == SHAMPOO_ROOTS_INT8_EMULATED && (slices < 4 || slices > kOzMaxSlices))
-    return fail(ctx, SHAMPOO_EINVAL, "slices must be in [4, 7]");
+    return fail(ctx, SHAMPOO_EINVAL, "slices must be in [4, 6]");
   if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "an asynchronous root job is in flight");
   ctx->root_method = method;
   if (method == SHAMPOO_ROOTS_INT8_EMULATED) ctx->oz_slices = slices;

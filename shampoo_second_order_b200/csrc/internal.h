@@ -113,9 +113,9 @@ struct NewtonWork {
 
 // Matrix sets sliced for the emulated products.
 enum : int { kOzX = 0, kOzT = 1, kOzT2 = 2, kOzT4 = 3, kOzM = 4, kOzSets = 5 };
-constexpr int kOzMaxSlices = 7;   // 7 accumulators of 64 TMEM columns
+constexpr int kOzMaxSlices = 6;   // accumulators of 64 TMEM columns, rotating over 8 slots
 // TMA descriptors over the int8 slice planes [kOzSets * qs * qcap][S][S]
-// (128-byte swizzle, K-major): a  box 128 x 128 (row tile), b  box 128 x 64.
+// (64-byte swizzle, K-major): a  box 64 (K) x 128 rows, b  box 64 x 64 rows.
 struct OzakiMaps {
   CUtensorMap a, b;
 };

@@ -25,7 +25,7 @@
 //   ozaki_split  per row: exponent and qs int8 slice planes of a float64 iterate
 //   ozaki_gemm   persistent, warp-specialised: lane 0 of warp 0 loads the
 //                slice planes by TMA (a stage = one slice of A's 128-row
-//                tile and of B's 64-row tile over 128 K), lane 0 of warp 1
+//                tile and of B's 64-row tile over 64 K), lane 0 of warp 1
 //                issues the int8 MMAs of every pair as soon as its slices
 //                are in, warps 2-5 combine the accumulators in float64, scale
 //                them and run the step's epilogue.
@@ -42,11 +42,16 @@ namespace {
 
 enum : int { kRunning = 0, kFinal = 4 };    // NewtonWork.state values read here
 constexpr int kBadExp = 1 << 20;             // exponent of a row holding NaN or Inf
-constexpr int kTileM = 128, kTileN = 64, kKBytes = 128;
-constexpr int kABytes = kTileM * kKBytes;    // 16 KB: one slice of the row tile
-constexpr int kBBytes = kTileN * kKBytes;    // 8 KB: one slice of the column tile
+// A stage holds one slice of the 128-row A tile and of the 64-row B tile
+// over 64 K (64-byte swizzled rows): 12 KB.  A K chunk needs its QS stages
+// at once (slice 0 pairs with every other), so 18 stages keep two chunks of
+// look-ahead in flight.
+constexpr int kTileM = 128, kTileN = 64, kKBytes = 64;
+constexpr int kABytes = kTileM * kKBytes;    // 8 KB
+constexpr int kBBytes = kTileN * kKBytes;    // 4 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kStages = 9;                   // one K chunk of 7 slices plus look-ahead
+constexpr int kStages = 18;
+constexpr int kSlots = 8;                    // TMEM accumulator slots of 64 columns (all 512)
 constexpr uint32_t kIdesc = tc::idesc_s8(kTileM, kTileN);
 
 // ---------------------------------------------------------------------------
@@ -184,19 +189,25 @@ __device__ __forceinline__ OzTile oz_decode(int t, const OzArgs& a) {
   return x;
 }
 
+// Power of two 2^e as a float64 (|e| well inside the normal range).
+__device__ __forceinline__ double pow2(int e) {
+  return __longlong_as_double(static_cast<long long>(1023 + e) << 52);
+}
+
+template <int QS>
 __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                                             const __grid_constant__ CUtensorMap map_b,
                                                             OzArgs args, int ntiles) {
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = args.S, qs = args.w.qs, qcap = args.w.qcap;
+  const int S = args.S, qcap = args.w.qcap;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;    // accumulators ready for the epilogue
-  uint64_t* tempty = tfull + 1;         // accumulators read out by the epilogue
-  uint64_t* drain = tempty + 1;
+  uint64_t* tfull = empty + kStages;    // [2] a tile's accumulators complete
+  uint64_t* sfree = tfull + 2;          // [kSlots] TMEM slot read out by the epilogue
+  uint64_t* drain = sfree + kSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -205,8 +216,9 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    tc::mbar_init(tfull, 1);
-    tc::mbar_init(tempty, 128);
+    tc::mbar_init(&tfull[0], 1);
+    tc::mbar_init(&tfull[1], 1);
+    for (int s = 0; s < kSlots; ++s) tc::mbar_init(&sfree[s], 128);
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -222,15 +234,16 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
-    int g = 0;
+    int s = 0;
+    uint32_t ph = 0;      // phase of the ring's current lap
+    bool first = true;    // the first lap needs no free stage
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       const OzTile x = oz_decode(t, args);
       if (x.skip) continue;
       bool ok = true;
       for (int kc = 0; kc < nk && ok; ++kc)
-        for (int k = 0; k < qs; ++k, ++g) {
-          const int s = g % kStages;
-          if (g >= kStages && !tc::mbar_wait(&empty[s], ((g / kStages) - 1) & 1)) {
+        for (int k = 0; k < QS; ++k) {
+          if (!first && !tc::mbar_wait(&empty[s], ph ^ 1)) {
             *abort_flag = 1;
             atomicExch(args.err, tc::kErrTimeout);
             ok = false;
@@ -238,61 +251,84 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
           }
           uint8_t* st = smem + s * kStageBytes;
           tc::mbar_expect_tx(&full[s], kStageBytes);
-          tc::tma_load_3d(st, &map_a, &full[s], kc * kKBytes, x.i0, (x.setA * qs + k) * qcap + x.m);
-          tc::tma_load_3d(st + kABytes, &map_b, &full[s], kc * kKBytes, x.j0, (x.setB * qs + k) * qcap + x.m);
+          tc::tma_load_3d(st, &map_a, &full[s], kc * kKBytes, x.i0, (x.setA * QS + k) * qcap + x.m);
+          tc::tma_load_3d(st + kABytes, &map_b, &full[s], kc * kKBytes, x.j0, (x.setB * QS + k) * qcap + x.m);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+            first = false;
+          }
         }
       if (!ok) break;
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
-    int g = 0, i = 0;
+    // Accumulator d of the i-th tile lives in TMEM slot (i QS + d) mod kSlots:
+    // the next tile starts in the slots its predecessor left free and waits
+    // for each other slot only when it first writes it.
+    int s = 0, i = 0;
+    uint32_t ph = 0;
+    const uint64_t desc0 = tc::smem_desc(0, 16, 512, 4);   // 64-byte swizzle; + (address >> 4)
+    const uint32_t ring = tc::smem_u32(smem);
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       const OzTile x = oz_decode(t, args);
       if (x.skip) continue;
-      if (i >= 1 && !tc::mbar_wait(tempty, (i - 1) & 1)) {
-        *abort_flag = 1;
-        atomicExch(args.err, tc::kErrTimeout);
-        break;
-      }
-      tc::fence_after_sync();
-      uint32_t inited = 0;   // accumulators written in this tile
+      const int g0 = i * QS;
       bool ok = true;
-      const uint32_t ring = tc::smem_u32(smem);
       for (int kc = 0; kc < nk && ok; ++kc) {
-        const int g0 = g;   // ring position of this chunk's slice 0
-        for (int k = 0; k < qs; ++k, ++g) {
-          const int s = g % kStages;
-          if (!tc::mbar_wait(&full[s], (g / kStages) & 1)) {
-            *abort_flag = 1;
-            atomicExch(args.err, tc::kErrTimeout);
+        int idx[QS];          // ring stage of each slice of this K chunk
+#pragma unroll
+        for (int k = 0; k < QS; ++k) {
+          if (!tc::mbar_wait(&full[s], ph)) {
             ok = false;
             break;
           }
-          tc::fence_after_sync();
-          // every pair (a, b), a + b <= qs - 1 (0-based), whose later slice is k
-          for (int o = 0; o <= k && o + k <= qs - 1; ++o) {
-            for (int sw = 0; sw < (o < k ? 2 : 1); ++sw) {   // (k, o), then (o, k) for o < k
-              const int ia = sw ? o : k, ib = sw ? k : o;
-              const int d = ia + ib;
-              const uint32_t dt = tmem + d * kTileN;
-              const uint32_t sa = ring + ((g0 + ia) % kStages) * kStageBytes;
-              const uint32_t sb = ring + ((g0 + ib) % kStages) * kStageBytes + kABytes;
+          idx[k] = s;
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+          if (kc == 0) {   // first writes of accumulators 2k - 1 and 2k: their slots must be read out
 #pragma unroll
-              for (int kk = 0; kk < kKBytes / 32; ++kk) {
-                const uint64_t da = tc::smem_desc(sa + kk * 32, 16, 1024);
-                const uint64_t db = tc::smem_desc(sb + kk * 32, 16, 1024);
-                tc::mma_i8(dt, da, db, kIdesc, ((inited >> d) & 1u) | (kk > 0));
-              }
-              inited |= 1u << d;
+            for (int d = 2 * k - 1; d <= 2 * k; ++d) {
+              if (d < 0 || d >= QS) continue;
+              const int gd = g0 + d;
+              if (gd >= kSlots && !tc::mbar_wait(&sfree[gd % kSlots], ((gd / kSlots) - 1) & 1)) ok = false;
+            }
+            if (!ok) break;
+          }
+          tc::fence_after_sync();
+          // every pair (a, b), a + b <= QS - 1 (0-based), whose later slice is
+          // k: (k, o) and (o, k).  The pair with o = k or o = k - 1 is the
+          // first to reach its accumulator a + b in a tile.
+#pragma unroll
+          for (int o = 0; o <= k; ++o) {
+            if (o + k > QS - 1) continue;
+#pragma unroll
+            for (int sw = 0; sw < 2; ++sw) {
+              if (sw == 1 && o == k) continue;
+              const int ia = sw ? o : k, ib = sw ? k : o;
+              const uint32_t dt = tmem + ((g0 + ia + ib) % kSlots) * kTileN;
+              const uint64_t da = desc0 + ((ring + idx[ia] * kStageBytes) >> 4);
+              const uint64_t db = desc0 + ((ring + idx[ib] * kStageBytes + kABytes) >> 4);
+              const bool lead = sw == 0 && (o == k || o == k - 1);
+#pragma unroll
+              for (int kk = 0; kk < kKBytes / 32; ++kk)
+                tc::mma_i8(dt, da + 2 * kk, db + 2 * kk, kIdesc, (kc > 0 || kk > 0 || !lead) ? 1u : 0u);
             }
           }
         }
         if (!ok) break;
         // this chunk's stages are free once its MMAs have read them
-        for (int k = 0; k < qs; ++k) tc::mma_commit(&empty[(g - qs + k) % kStages]);
+#pragma unroll
+        for (int k = 0; k < QS; ++k) tc::mma_commit(&empty[idx[k]]);
       }
-      if (!ok) break;
-      tc::mma_commit(tfull);
+      if (!ok) {
+        *abort_flag = 1;
+        atomicExch(args.err, tc::kErrTimeout);
+        break;
+      }
+      tc::mma_commit(&tfull[i & 1]);
       ++i;
     }
     tc::mma_commit(drain);
@@ -305,7 +341,7 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       const OzTile x = oz_decode(t, args);
       if (x.skip) continue;
-      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tfull, i & 1) && !*abort_flag);
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&tfull[i & 1], (i >> 1) & 1) && !*abort_flag);
       if (!ok) {
         if (lane == 0) {
           *abort_flag = 1;
@@ -316,21 +352,25 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
       tc::fence_after_sync();
       const int m = x.m, rl = q * 32 + lane, r = x.i0 + rl;
       const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-      double acc[2][32];
+      // Accumulator d weighs 2^{-7(d+2)}: the value is 2^{-7(QS+1)} times the
+      // exact int64 sum of acc_d 2^{7(QS-1-d)} (below 2^60 for S <= 1024).
+      // Each slot is released as soon as it is read.
+      long long tot[64];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int j = 0; j < 64; ++j) tot[j] = 0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[c][j] = 0.0;
-        for (int d = 0; d < qs; ++d) {
+      for (int d = 0; d < QS; ++d) {
+        const int slot = (i * QS + d) % kSlots;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           float v[32];
-          tc::tmem_ld32(trow + d * kTileN + c * 32, v);
-          const double wd = ldexp(1.0, -7 * (d + 2));
+          tc::tmem_ld32(trow + slot * kTileN + c * 32, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c][j] = fma((double)__float_as_int(v[j]), wd, acc[c][j]);
+          for (int j = 0; j < 32; ++j) tot[c * 32 + j] += (long long)__float_as_int(v[j]) << (7 * (QS - 1 - d));
         }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&sfree[slot]);
       }
-      tc::fence_before_sync();
-      tc::mbar_arrive(tempty);   // the next tile's MMAs may overwrite the accumulators
       ++i;
 
       const size_t base = (size_t)m * S * S;
@@ -354,31 +394,46 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
       const bool resid = args.step == 2;
       const double sn = resid ? newton_sched(w, m, args.it + 1) : 0.0, pinv = 1.0 / p;
       const int n = args.mats[m].size;
+      // whole tile strictly above the diagonal: every entry is stored and mirrored
+      const bool above = x.j0 >= x.i0 + kTileM;
       double dev = 0.0, f2 = 0.0;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int col = x.j0 + c * 32 + j;
-          if (r >= S || col >= S || r > col) continue;
-          const int e2 = eb[col];
-          const double v = (ea == kBadExp || e2 == kBadExp) ? __longlong_as_double(0x7ff8000000000000ll)
-                                                          : ldexp(acc[c][j], ea + e2) * mul;
+      const double sc = mul * pow2(ea - 7 * (QS + 1));
+      // one entry (r, col) of the upper triangle: stored, mirrored and, for
+      // step C, folded into the residual and turned into the next T
+      auto emit = [&](int col, double v, bool stored) {
+        if (r >= S || col >= S || r > col) return;
+        if (!stored) {
           C[(size_t)r * S + col] = v;
           if (r < col) C[(size_t)col * S + r] = v;
-          if (resid) {
-            const double dl = (r == col) ? 1.0 : 0.0;
-            if (r < n && col < n) {
-              double xd = fabs(v - dl);
-              if (!(xd <= DBL_MAX)) xd = INFINITY;
-              dev = fmax(dev, xd);
-              f2 += (r == col ? 1.0 : 2.0) * xd * xd;   // an entry above the diagonal counts for its mirror too
-            }
-            const double tn = ((p + 1) * dl - sn * v) * pinv;   // next T = ((p+1) I - s_{k+1} M_next) / p
-            w.T[base + (size_t)r * S + col] = tn;
-            if (r < col) w.T[base + (size_t)col * S + r] = tn;
-          }
         }
+        if (resid) {
+          const double dl = (r == col) ? 1.0 : 0.0;
+          if (r < n && col < n) {
+            double xd = fabs(v - dl);
+            if (!(xd <= DBL_MAX)) xd = INFINITY;
+            dev = fmax(dev, xd);
+            f2 += (r == col ? 1.0 : 2.0) * xd * xd;   // an entry above the diagonal counts for its mirror too
+          }
+          const double tn = ((p + 1) * dl - sn * v) * pinv;   // next T = ((p+1) I - s_{k+1} M_next) / p
+          w.T[base + (size_t)r * S + col] = tn;
+          if (r < col) w.T[base + (size_t)col * S + r] = tn;
+        }
+      };
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) {
+        const int col = x.j0 + j;
+        const int e0 = eb[col], e1 = eb[col + 1];
+        const bool bad0 = ea == kBadExp || e0 == kBadExp, bad1 = ea == kBadExp || e1 == kBadExp;
+        const double nan = __longlong_as_double(0x7ff8000000000000ll);
+        const double v0 = bad0 ? nan : (double)tot[j] * (sc * pow2(e0));
+        const double v1 = bad1 ? nan : (double)tot[j + 1] * (sc * pow2(e1));
+        if (above && r < S) {
+          *reinterpret_cast<double2*>(C + (size_t)r * S + col) = make_double2(v0, v1);
+          C[(size_t)col * S + r] = v0;
+          C[(size_t)(col + 1) * S + r] = v1;
+        }
+        emit(col, v0, above);
+        emit(col + 1, v1, above);
       }
       if (resid) {
         dev = warp_max(dev);
@@ -407,6 +462,18 @@ int sm_count_oz() {
   return n;
 }
 
+template <int QS>
+cudaError_t launch_gemm(const OzakiMaps& maps, const OzArgs& a, int ntiles, int grid, int smem, cudaStream_t s) {
+  static bool configured = false;   // the attribute is per instantiation
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(ozaki_gemm_kernel<QS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  ozaki_gemm_kernel<QS><<<grid, 192, smem, s>>>(maps.a, maps.b, a, ntiles);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_ozaki_split(const NewtonMat* mats, int nm, int S, int it, unsigned sets, NewtonWork w,
@@ -431,19 +498,17 @@ cudaError_t launch_ozaki_split(const NewtonMat* mats, int nm, int S, int it, uns
 
 cudaError_t launch_ozaki_step(const OzakiMaps& maps, int step, const NewtonMat* mats, int nm, int S, int it,
                               NewtonWork w, int* err, cudaStream_t s) {
-  static bool configured = false;
-  const int smem = kStages * kStageBytes + 1024 + 256;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(ozaki_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  const int smem = kStages * kStageBytes + 1024 + 512;   // ring, alignment slack, barriers
   OzArgs a{};
   a.mats = mats; a.w = w; a.S = S; a.it = it; a.step = step; a.ntri = oz_ntri(S); a.err = err;
   const int ntiles = nm * (step == 0 ? 2 : 1) * a.ntri;
   const int grid = ntiles < sm_count_oz() ? ntiles : sm_count_oz();
-  ozaki_gemm_kernel<<<grid, 192, smem, s>>>(maps.a, maps.b, a, ntiles);
-  return cudaGetLastError();
+  switch (w.qs) {
+    case 4: return launch_gemm<4>(maps, a, ntiles, grid, smem, s);
+    case 5: return launch_gemm<5>(maps, a, ntiles, grid, smem, s);
+    case 6: return launch_gemm<6>(maps, a, ntiles, grid, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace shampoo
