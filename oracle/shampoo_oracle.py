@@ -24,7 +24,8 @@ Optimization for Deep Learning", Anil, Gupta, Koren, Regan, Singer):
 * segment 14: the roots L^{-1/4}, R^{-1/4} are recomputed only every so many
   steps; stale roots are used in between.
 * segment 16: large layers are split into blocks, each preconditioned on its
-  own (Lemma 2).
+  own (Lemma 2); for a layer too large even for that (a big embedding or
+  softmax), only one of L and R is kept (Lemma 1).
 
 The pages print no formula, constant or worked example.  Where they are
 silent this module takes the plainest reading, listed here once:
@@ -42,6 +43,10 @@ silent this module takes the plainest reading, listed here once:
   D = g / sqrt(a + eps), s = ||D||_F / ||P||_F over the whole parameter
   (s = 0 when ||P||_F = 0), update U = s * P.
 * momentum (heavy ball, m0 = 0): m <- mu*m + U; W <- W - lr*m.
+* one-sided blocks (Lemma 1): the kept factor is accumulated as above and
+  taken to the power -2/p (-1/2 for p = 4: full-matrix Adagrad along that
+  dimension, the exponent of the 1-D case); the dropped factor is never
+  accumulated and its root is the identity, so P = L^{-2/p} G or G R^{-2/p}.
 * roots are first computed after the first statistics update and then at the
   caller's interval; apply never runs without roots.
 * a gradient holding a NaN or an infinity leaves its parameter untouched for
@@ -53,6 +58,9 @@ import numpy as np
 
 GRAFT_NONE = 0
 GRAFT_ADAGRAD = 1
+SIDES_BOTH = 0     # L and R
+SIDE_LEFT = 1      # L only (Lemma 1)
+SIDE_RIGHT = 2     # R only (Lemma 1)
 
 
 # ---------------------------------------------------------------------------
@@ -150,13 +158,14 @@ class ShampooOracle:
     """Blocked Shampoo with layer-wise Adagrad grafting, all in float64.
 
     ``shapes`` is a list of (rows, cols) for 2-D parameters and (n,) for 1-D
-    ones.  State persists across calls; one optimizer step is
-    ``update_stats(grads)``, then ``compute_roots()`` on root steps, then
-    ``apply(params, grads, lr)``.
+    ones.  ``sides`` (optional) gives per parameter SIDES_BOTH, SIDE_LEFT or
+    SIDE_RIGHT (2-D parameters only).  State persists across calls; one
+    optimizer step is ``update_stats(grads)``, then ``compute_roots()`` on
+    root steps, then ``apply(params, grads, lr)``.
     """
 
     def __init__(self, shapes, block_size, beta2, eps, p=4,
-                 graft=GRAFT_ADAGRAD, momentum=0.0, root_route="eigh"):
+                 graft=GRAFT_ADAGRAD, momentum=0.0, root_route="eigh", sides=None):
         self.shapes = [tuple(int(d) for d in s) for s in shapes]
         self.b = int(block_size)
         self.beta2 = float(beta2)
@@ -165,6 +174,7 @@ class ShampooOracle:
         self.graft = int(graft)
         self.mu = float(momentum)
         self.root_route = root_route
+        self.sides = [SIDES_BOTH] * len(self.shapes) if sides is None else [int(x) for x in sides]
         self.blocks = []      # per param: list of block tuples
         self.stats = []       # per param: list of (L, R) or [S]
         self.roots = []       # per param: list of (Lr, Rr) or [Sr], or None
@@ -196,11 +206,15 @@ class ShampooOracle:
                 self.skipped.add(i)
                 continue
             if len(s) == 2:
+                side = self.sides[i]
                 for k, (r0, c0, m, n) in enumerate(self.blocks[i]):
                     G = g[r0:r0 + m, c0:c0 + n]
                     L, R = self.stats[i][k]
-                    self.stats[i][k] = (self.beta2 * L + G @ G.T,
-                                        self.beta2 * R + G.T @ G)
+                    if side != SIDE_RIGHT:
+                        L = self.beta2 * L + G @ G.T
+                    if side != SIDE_LEFT:
+                        R = self.beta2 * R + G.T @ G
+                    self.stats[i][k] = (L, R)
             else:
                 for k, (s0, ln) in enumerate(self.blocks[i]):
                     v = g[s0:s0 + ln].reshape(ln, 1)
@@ -220,8 +234,14 @@ class ShampooOracle:
         p2 = self.p / 2.0
         for i, s in enumerate(self.shapes):
             if len(s) == 2:
-                self.roots[i] = [(self._root(L, self.p), self._root(R, self.p))
-                                 for (L, R) in self.stats[i]]
+                side = self.sides[i]
+                if side == SIDE_LEFT:
+                    self.roots[i] = [(self._root(L, p2), np.eye(R.shape[0])) for (L, R) in self.stats[i]]
+                elif side == SIDE_RIGHT:
+                    self.roots[i] = [(np.eye(L.shape[0]), self._root(R, p2)) for (L, R) in self.stats[i]]
+                else:
+                    self.roots[i] = [(self._root(L, self.p), self._root(R, self.p))
+                                     for (L, R) in self.stats[i]]
             else:
                 self.roots[i] = [self._root(S, p2) for S in self.stats[i]]
 
@@ -275,9 +295,12 @@ class ShampooOracle:
         mats = []
         for i, s in enumerate(self.shapes):
             if len(s) == 2:
+                side = self.sides[i]
+                pl = {SIDES_BOTH: self.p, SIDE_LEFT: self.p / 2.0, SIDE_RIGHT: 0}[side]
+                pr = {SIDES_BOTH: self.p, SIDE_LEFT: 0, SIDE_RIGHT: self.p / 2.0}[side]
                 for (L, R) in self.stats[i]:
-                    mats.append((L, self.p))
-                    mats.append((R, self.p))
+                    mats.append((L, pl))      # exponent 0: a dropped factor, root I
+                    mats.append((R, pr))
         for i, s in enumerate(self.shapes):
             if len(s) == 1:
                 for S in self.stats[i]:

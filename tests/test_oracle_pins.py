@@ -13,8 +13,8 @@ import os
 import numpy as np
 import pytest
 
-from oracle import (GRAFT_ADAGRAD, GRAFT_NONE, ShampooOracle, block_partition,
-                    coupled_newton_inverse_root, inverse_root, vector_segments)
+from oracle import (GRAFT_ADAGRAD, GRAFT_NONE, SIDE_LEFT, SIDE_RIGHT, ShampooOracle,
+                    block_partition, coupled_newton_inverse_root, inverse_root, vector_segments)
 from shampoo_second_order_b200 import workloads as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -380,3 +380,77 @@ def test_spd_batch_spectrum():
         assert np.allclose(np.sort(ev), np.sort(lam[i]), rtol=1e-8)
     assert abs(lam[0].max() / lam[0].min() - 1e2) < 1e-6
     assert abs(lam[2].max() / lam[2].min() - 1e6) < 1e-2
+
+
+# --------------------------------------------------------------------------
+# One-sided preconditioning (segment 16, Lemma 1)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("side", [SIDE_LEFT, SIDE_RIGHT])
+@pytest.mark.parametrize("shape", [(4, 6), (6, 4)])
+def test_one_sided_rank_one_closed_form(side, shape):
+    """One step with G = u v^T, one factor only: the kept factor has the
+    eigenvalue |u|^2 |v|^2 along G's direction, so its -1/2 power gives
+    G / sqrt(|G|^2 + eps) -- the two-sided result, while a -1/4 power or a
+    root of the never-accumulated factor would not."""
+    rng = np.random.default_rng(11)
+    u, v = rng.standard_normal(shape[0]), rng.standard_normal(shape[1])
+    G = np.outer(u, v)
+    eps = 1e-4
+    o = ShampooOracle([shape], 64, 1.0, eps, graft=GRAFT_NONE, sides=[side])
+    Wn = o.step([np.zeros(shape)], [G], 1.0, do_roots=True)[0]
+    assert np.allclose(Wn, -G / np.sqrt(np.sum(G * G) + eps), rtol=1e-11, atol=1e-14)
+
+
+def test_one_sided_right_disjoint_columns_closed_form():
+    """Right factor only, each step's gradient non-zero in one column c_t:
+    R = sum_t beta2^(T-t) |x_t|^2 e_c e_c^T is diagonal, so the last step is
+    column c_T divided by sqrt(R[c_T, c_T] + eps)."""
+    rng = np.random.default_rng(12)
+    m, n, beta2, eps = 5, 4, 0.9, 1e-3
+    cols = [0, 2, 0, 3, 2, 0]
+    xs = [rng.standard_normal(m) for _ in cols]
+    o = ShampooOracle([(m, n)], 64, beta2, eps, graft=GRAFT_NONE, sides=[SIDE_RIGHT])
+    W = np.zeros((m, n))
+    for c, x in zip(cols, xs):
+        G = np.zeros((m, n))
+        G[:, c] = x
+        Wn = o.step([W], [G], 1.0, do_roots=True)[0]
+        W, dW = Wn, Wn - W
+    T = len(cols)
+    r = sum(beta2 ** (T - 1 - t) * (xs[t] @ xs[t]) for t in range(T) if cols[t] == cols[-1])
+    ref = np.zeros((m, n))
+    ref[:, cols[-1]] = -xs[-1] / np.sqrt(r + eps)
+    assert np.allclose(dW, ref, rtol=1e-11, atol=1e-14)
+
+
+def test_one_sided_left_column_is_full_matrix_adagrad_on_the_vector():
+    """A 2-D m x 1 parameter with only L kept is full-matrix Adagrad on the
+    column, which is what the 1-D path does: both give the same weights over
+    several grafted momentum steps."""
+    rng = np.random.default_rng(13)
+    m = 7
+    a = ShampooOracle([(m, 1)], 64, 0.95, 1e-4, momentum=0.5, sides=[SIDE_LEFT])
+    b = ShampooOracle([(m,)], 64, 0.95, 1e-4, momentum=0.5)
+    Wa, Wb = [rng.standard_normal((m, 1))], [None]
+    Wb = [Wa[0][:, 0].copy()]
+    for t in range(5):
+        g = rng.standard_normal(m)
+        Wa = a.step(Wa, [g.reshape(m, 1)], 0.1, do_roots=(t % 2 == 0))
+        Wb = b.step(Wb, [g], 0.1, do_roots=(t % 2 == 0))
+        assert np.allclose(Wa[0][:, 0], Wb[0], rtol=1e-12, atol=1e-15)
+
+
+def test_one_sided_dropped_factor_stays_zero_with_identity_root():
+    rng = np.random.default_rng(14)
+    o = ShampooOracle([(6, 9), (9, 6)], 4, 0.9, 1e-6, sides=[SIDE_LEFT, SIDE_RIGHT])
+    for _ in range(2):
+        o.update_stats([rng.standard_normal((6, 9)), rng.standard_normal((9, 6))])
+    o.compute_roots()
+    for (L, R), (Lr, Rr) in zip(o.stats[0], o.roots[0]):
+        assert not R.any() and np.array_equal(Rr, np.eye(R.shape[0]))
+        assert np.allclose(Lr, inverse_root(L, 1e-6, 2.0), rtol=1e-12)
+    for (L, R), (Lr, Rr) in zip(o.stats[1], o.roots[1]):
+        assert not L.any() and np.array_equal(Lr, np.eye(L.shape[0]))
+        assert np.allclose(Rr, inverse_root(R, 1e-6, 2.0), rtol=1e-12)
+    exps = [e for _, e in o.matrices()]
+    assert exps[:4] == [2.0, 0, 2.0, 0] and exps[-2:] == [0, 2.0]
