@@ -60,6 +60,12 @@ typedef enum {
 } shampoo_graft;
 
 typedef enum {
+  SHAMPOO_SIDES_BOTH = 0,     /* L and R (the default)                         */
+  SHAMPOO_SIDE_LEFT = 1,      /* L only: P = L^{-2/p} G                        */
+  SHAMPOO_SIDE_RIGHT = 2      /* R only: P = G R^{-2/p}                        */
+} shampoo_side;
+
+typedef enum {
   SHAMPOO_ROOTS_FP64 = 0,          /* Newton products in float64 (mma f64)     */
   SHAMPOO_ROOTS_INT8_EMULATED = 1  /* the same products emulated on the int8
                                       tensor cores (Ozaki scheme)              */
@@ -231,6 +237,22 @@ shampoo_status shampoo_set_root_options(shampoo_ctx* ctx, double tol, int max_it
 shampoo_status shampoo_set_root_method(shampoo_ctx* ctx, int method, int slices);
 
 /*
+ * shampoo_set_one_sided -- keep only one factor for every block of 2-D
+ * parameter `param` (podcast transcript, segment 16: for a layer too large
+ * even when blocked, such as a big embedding or softmax, only L or only R is
+ * used, Lemma 1).  The kept factor is accumulated as usual and rooted at
+ * exponent -2/p (-1/2 for p = 4: full-matrix Adagrad along that dimension);
+ * the dropped factor is never accumulated, never rooted, and its root slot
+ * holds the identity, so the apply computes P = L^{-1/2} G (side LEFT) or
+ * P = G R^{-1/2} (side RIGHT).  SHAMPOO_SIDES_BOTH restores the default.
+ * Call between shampoo_create and the first shampoo_update_stats
+ * (SHAMPOO_ESTATE later).  SHAMPOO_EINVAL for a 1-D parameter, a bad index
+ * or side, or a context created with p != 4.  Synchronises the stream.
+ * shampoo_matrix_info reports root_p = 0 for a dropped factor.
+ */
+shampoo_status shampoo_set_one_sided(shampoo_ctx* ctx, int param, int side);
+
+/*
  * shampoo_num_matrices -- number of statistics matrices: 2 per 2-D block
  * (L then R, blocks in parameter order, row-major within a parameter), then
  * 1 per 1-D segment (parameter order).  Each lives in a b x b slot.
@@ -240,7 +262,8 @@ int shampoo_num_matrices(const shampoo_ctx* ctx);
 /*
  * shampoo_matrix_info -- for statistic `index`: its valid side (the block's
  * rows for L, columns for R, the segment length for S) and its root exponent
- * denominator (p, or p/2 for a segment).  Host values.
+ * denominator (p, or p/2 for a segment or a one-sided block's kept factor,
+ * 0 for its dropped factor).  Host values.
  */
 shampoo_status shampoo_matrix_info(const shampoo_ctx* ctx, int index,
                                    int* size, int* root_p);

@@ -15,6 +15,7 @@ STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ENOMEM", 3: "ECUDA", 4: "ENONFINITE",
                 5: "ENOTCONVERGED", 6: "ESTATE", 7: "EBUSY"}
 GRAFT_NONE, GRAFT_ADAGRAD = 0, 1
 ROOTS_FP64, ROOTS_INT8_EMULATED = 0, 1
+SIDES_BOTH, SIDE_LEFT, SIDE_RIGHT = 0, 1, 2
 F32, BF16 = 0, 1
 
 # name -> (restype, argtypes), exactly the declarations of include/shampoo.h
@@ -32,6 +33,7 @@ SIGNATURES = {
     "shampoo_nonfinite_status": (C.c_int, [_P, C.POINTER(C.c_int)]),
     "shampoo_set_root_options": (C.c_int, [_P, C.c_double, C.c_int]),
     "shampoo_set_root_method": (C.c_int, [_P, C.c_int, C.c_int]),
+    "shampoo_set_one_sided": (C.c_int, [_P, C.c_int, C.c_int]),
     "shampoo_num_matrices": (C.c_int, [_P]),
     "shampoo_matrix_info": (C.c_int, [_P, C.c_int, C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "shampoo_read_matrix": (C.c_int, [_P, C.c_int, C.c_int, _P]),
@@ -156,6 +158,10 @@ def shampoo_set_root_options(ctx, tol, max_iters):
 
 def shampoo_set_root_method(ctx, method, slices=6):
     return _check(lib().shampoo_set_root_method(ctx, int(method), int(slices)), ctx)
+
+
+def shampoo_set_one_sided(ctx, param, side):
+    return _check(lib().shampoo_set_one_sided(ctx, int(param), int(side)), ctx)
 
 
 def shampoo_num_matrices(ctx):

@@ -134,7 +134,9 @@ struct shampoo_ctx {
   std::vector<SegDesc> segs;
   std::vector<ChunkDesc> chunks;
   std::vector<ChunkDesc> chunks1d;   // chunks of the 1-D parameters only
-  std::vector<NewtonMat> mats;
+  std::vector<NewtonMat> mats;       // per statistic slot (p = 0: a dropped one-sided factor)
+  std::vector<NewtonMat> run_mats;   // the slots the root computation runs on
+  std::vector<int> param_side;       // per parameter: 0 both factors, 1 L only, 2 R only
   int64_t total = 0;
   int nmat = 0;
 
@@ -144,7 +146,7 @@ struct shampoo_ctx {
   SegDesc* d_segs = nullptr;
   ChunkDesc* d_chunks = nullptr;
   ChunkDesc* d_chunks1d = nullptr;
-  NewtonMat* d_mats = nullptr;
+  NewtonMat* d_mats = nullptr;       // device copy of run_mats
   const void** d_gptr = nullptr;
   float** d_wptr = nullptr;
   float* stats = nullptr;
@@ -491,7 +493,7 @@ shampoo_status run_root_job(shampoo_ctx* o, shampoo_ctx* ctx, double tol, int ma
   // a matrix that does not converge keeps the root in use
   CK(cudaMemcpyAsync(o->roots_back, o->roots, (size_t)o->nmat * slot * sizeof(float),
                      cudaMemcpyDeviceToDevice, st));
-  shampoo_status r = run_newton(ctx, &o->prof, o->mats, o->d_mats, o->d_retry, o->stats_snap, slot, o->S, 1,
+  shampoo_status r = run_newton(ctx, &o->prof, o->run_mats, o->d_mats, o->d_retry, o->stats_snap, slot, o->S, 1,
                                 o->roots_back, slot, o->S, o->S, o->eps, tol, max_iters,
                                 o->newton_chunk, o->nw, o->has_root, nullptr, o->h_count, o->ev, st, nf,
                                 mi, iters, use_oz ? &o->oz : nullptr, o->d_err);
@@ -677,7 +679,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
     if (nd == 2) {
       for (int64_t r0 = 0; r0 < r; r0 += b)
         for (int64_t c0 = 0; c0 < c; c0 += b) {
-          BlockDesc bd;
+          BlockDesc bd{};
           bd.param = i;
           bd.r0 = r0;
           bd.c0 = c0;
@@ -714,6 +716,8 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   for (size_t k = 0; k < ctx->segs.size(); ++k)
     ctx->mats.push_back({mat0 + (int)k, ctx->segs[k].len, p / 2, 0});
   ctx->nmat = (int)ctx->mats.size();
+  ctx->run_mats = ctx->mats;
+  ctx->param_side.assign(nparams, 0);
 
   shampoo_status st;
   if ((st = upload(ctx, &ctx->d_params, ctx->params)) != SHAMPOO_OK ||
@@ -721,7 +725,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
       (st = upload(ctx, &ctx->d_segs, ctx->segs)) != SHAMPOO_OK ||
       (st = upload(ctx, &ctx->d_chunks, ctx->chunks)) != SHAMPOO_OK ||
       (st = upload(ctx, &ctx->d_chunks1d, ctx->chunks1d)) != SHAMPOO_OK ||
-      (st = upload(ctx, &ctx->d_mats, ctx->mats)) != SHAMPOO_OK) {
+      (st = upload(ctx, &ctx->d_mats, ctx->run_mats)) != SHAMPOO_OK) {
     g_create_err = ctx->err;
     shampoo_destroy(ctx);
     return st;
@@ -847,7 +851,7 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
     if (os != SHAMPOO_OK) return os;
     ctx->nw.qs = ctx->oz_slices;
   }
-  shampoo_status st = run_newton(ctx, &ctx->prof, ctx->mats, ctx->d_mats, ctx->d_retry, ctx->stats,
+  shampoo_status st = run_newton(ctx, &ctx->prof, ctx->run_mats, ctx->d_mats, ctx->d_retry, ctx->stats,
                                  slot, ctx->S, 1,
                                  ctx->roots, slot, ctx->S, ctx->S, ctx->eps, ctx->tol,
                                  ctx->max_iters, ctx->newton_chunk, ctx->nw, ctx->has_root, nullptr,
@@ -1003,6 +1007,45 @@ shampoo_status shampoo_set_root_method(shampoo_ctx* ctx, int method, int slices)
   return SHAMPOO_OK;
 }
 
+shampoo_status shampoo_set_one_sided(shampoo_ctx* ctx, int param, int side) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (param < 0 || param >= ctx->nparams || side < SHAMPOO_SIDES_BOTH || side > SHAMPOO_SIDE_RIGHT)
+    return fail(ctx, SHAMPOO_EINVAL, "bad parameter index or side");
+  if (ctx->ndim[param] != 2) return fail(ctx, SHAMPOO_EINVAL, "a 1-D parameter has a single factor already");
+  if (ctx->p != 4) return fail(ctx, SHAMPOO_EINVAL, "one-sided blocks need p = 4 (the kept factor is rooted at p/2)");
+  if (ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "set_one_sided after the first update_stats");
+  const int S = ctx->S, p = ctx->p;
+  ctx->param_side[param] = side;
+  std::vector<float> eye;
+  for (size_t k = 0; k < ctx->blocks.size(); ++k) {
+    BlockDesc& bd = ctx->blocks[k];
+    if (bd.param != param) continue;
+    bd.side = side;
+    ctx->mats[2 * k].p = side == SHAMPOO_SIDE_RIGHT ? 0 : (side == SHAMPOO_SIDE_LEFT ? p / 2 : p);
+    ctx->mats[2 * k + 1].p = side == SHAMPOO_SIDE_LEFT ? 0 : (side == SHAMPOO_SIDE_RIGHT ? p / 2 : p);
+    // the dropped factor's root is the identity on its valid corner
+    for (int h = 0; h < 2; ++h) {
+      if (ctx->mats[2 * k + h].p != 0) continue;
+      const int n = ctx->mats[2 * k + h].size;
+      eye.assign((size_t)S * S, 0.f);
+      for (int d = 0; d < n; ++d) eye[(size_t)d * S + d] = 1.f;
+      CK(cudaMemcpy(ctx->roots + (size_t)(2 * k + h) * S * S, eye.data(), eye.size() * sizeof(float),
+                    cudaMemcpyHostToDevice));
+    }
+  }
+  ctx->run_mats.clear();
+  for (const auto& m : ctx->mats)
+    if (m.p > 0) ctx->run_mats.push_back(m);
+  if (!ctx->blocks.empty())
+    CK(cudaMemcpy(ctx->d_blocks, ctx->blocks.data(), ctx->blocks.size() * sizeof(BlockDesc), cudaMemcpyHostToDevice));
+  if (!ctx->run_mats.empty())
+    CK(cudaMemcpy(ctx->d_mats, ctx->run_mats.data(), ctx->run_mats.size() * sizeof(NewtonMat),
+                  cudaMemcpyHostToDevice));
+  CK(launch_split(ctx->roots, (int64_t)ctx->nmat * S * S, ctx->rplanes, ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  return SHAMPOO_OK;
+}
+
 int shampoo_num_matrices(const shampoo_ctx* ctx) { return ctx ? ctx->nmat : 0; }
 
 shampoo_status shampoo_matrix_info(const shampoo_ctx* ctx, int index, int* size, int* root_p) {
@@ -1035,7 +1078,9 @@ shampoo_status shampoo_read_matrix(shampoo_ctx* ctx, int which, int index, float
 shampoo_status shampoo_root_iterations(shampoo_ctx* ctx, int32_t* out) {
   if (!ctx || !out) return fail(ctx, SHAMPOO_EINVAL, "ctx or out is NULL");
   if (ctx->root_iters.empty()) return fail(ctx, SHAMPOO_ESTATE, "no roots computed yet");
-  std::memcpy(out, ctx->root_iters.data(), ctx->root_iters.size() * sizeof(int32_t));
+  // slots past the last one iterated (dropped one-sided factors) report 0
+  std::memset(out, 0, ctx->nmat * sizeof(int32_t));
+  std::memcpy(out, ctx->root_iters.data(), std::min<size_t>(ctx->root_iters.size(), ctx->nmat) * sizeof(int32_t));
   return SHAMPOO_OK;
 }
 

@@ -10,6 +10,7 @@ namespace shampoo {
 struct BlockDesc {
   int param;     // parameter index
   int m, n;      // valid rows / cols of the block
+  int side;      // factors kept: 0 both, 1 L only, 2 R only (one-sided, Lemma 1)
   int64_t r0, c0;  // top-left element in the parameter
   int64_t ld;    // the parameter's row length (cols)
 };

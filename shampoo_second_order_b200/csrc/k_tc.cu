@@ -95,6 +95,8 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const TcArgs& a) {
     x.skip = x.i0 >= bd.m || x.j0 >= bd.n;
     x.K = (MODE == kApplyY) ? bd.n : bd.m;
   }
+  // a one-sided block never accumulates its dropped factor
+  if (MODE == kStats) x.skip = x.skip || (bd.side == 1 && x.isR) || (bd.side == 2 && !x.isR);
   x.skip = x.skip || a.flags[bd.param] != 0;
   return x;
 }

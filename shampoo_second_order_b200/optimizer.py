@@ -82,6 +82,11 @@ class Shampoo:
         emulated on the int8 tensor cores with `slices` 7-bit slices)."""
         L.shampoo_set_root_method(self.ctx, _METHODS[method], slices)
 
+    def set_one_sided(self, index, side):
+        """Keep only one factor ("left": L, "right": R, "both": the default)
+        for every block of 2-D parameter `index`; before the first step."""
+        L.shampoo_set_one_sided(self.ctx, index, _SIDES[side])
+
     def root_iterations(self):
         return L.shampoo_root_iterations(self.ctx)
 
@@ -136,3 +141,4 @@ def batched_inverse_root(A, p, eps, tol=1e-6, max_iters=100, stream=None, method
 
 
 _METHODS = {"fp64": L.ROOTS_FP64, "int8": L.ROOTS_INT8_EMULATED}
+_SIDES = {"both": L.SIDES_BOTH, "left": L.SIDE_LEFT, "right": L.SIDE_RIGHT}

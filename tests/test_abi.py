@@ -85,6 +85,7 @@ def test_null_context_calls(lib):
     assert lib.shampoo_install_roots(None, 0, None) == L.EINVAL
     assert lib.shampoo_roots_generation(None) == -1
     assert lib.shampoo_set_root_method(None, 1, 6) == L.EINVAL
+    assert lib.shampoo_set_one_sided(None, 0, 1) == L.EINVAL
     lib.shampoo_destroy(None)
 
 

@@ -54,12 +54,19 @@ def pieces(shape, b):
     return [(slice(s0, s0 + ln),) for (s0, ln) in vector_segments(shape[0], b)]
 
 
+SIDE_CODE = {"both": 0, "left": 1, "right": 2}
+
+
 def run_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, interval, seed, gstd,
-             check_every=True, check_state=True, method="fp64"):
+             check_every=True, check_state=True, method="fp64", sides=None):
     from shampoo_second_order_b200 import Shampoo
-    o = ShampooOracle(shapes, b, beta2, eps, 4, graft, mu)
+    o = ShampooOracle(shapes, b, beta2, eps, 4, graft, mu,
+                      sides=None if sides is None else [SIDE_CODE[x] for x in sides])
     opt = Shampoo(shapes, b, beta2, eps, 4, graft, mu, gdtype)
     opt.set_root_method(method)
+    for i, sd in enumerate(sides or []):
+        if sd != "both":
+            opt.set_one_sided(i, sd)
     W0 = wl.make_params(shapes, seed)
     Wo = [w.astype(np.float64) for w in W0]
     Wd = [torch.from_numpy(w).cuda() for w in W0]
@@ -81,6 +88,7 @@ def run_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, interval, seed
             for k in range(opt.num_matrices()):
                 S, _ = opt.read_matrix(0, k)
                 worst["stats"] = max(worst["stats"], rel(S, mats[k][0]))
+                assert opt.matrix_info(k)[1] == mats[k][1]
                 ev = np.linalg.eigvalsh(mats[k][0]) + eps
                 if ev.max() / max(ev.min(), 1e-300) > 1e6:
                     continue
@@ -238,6 +246,44 @@ def test_transformer_layer_b512_int8_emulated_roots():
                  c["lr"], c["grad_dtype"], 21, c["root_interval"], c["seed"], c["grad_std"],
                  check_every=False, method="int8")
     assert_worst(w)
+
+
+# --------------------------------------------------------------------------
+# one-sided blocks (Lemma 1)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("gdtype,method", [("f32", "fp64"), ("bf16", "fp64"), ("f32", "int8")])
+def test_one_sided_ragged_set(gdtype, method):
+    shapes = [(200, 130), (64, 64), (19, 200), (130,), (300, 64), (1, 77)]
+    sides = ["left", "both", "right", "both", "right", "left"]
+    w = run_pair(shapes, 64, 0.99, 1e-6, 1, 0.9, 0.1, gdtype, steps=6, interval=3, seed=9,
+                 gstd=1e-2, method=method, sides=sides)
+    assert_worst(w)
+
+
+def test_one_sided_embedding_block_512():
+    """A tall embedding-like weight kept on its column side only (the
+    vocabulary side's statistics are never formed), bf16 gradients, b = 512."""
+    shapes = [(4096, 512), (512, 512)]
+    w = run_pair(shapes, 512, 0.999, 1e-6, 1, 0.0, 0.1, "bf16", steps=4, interval=2, seed=10,
+                 gstd=1e-3, check_every=False, sides=["right", "both"])
+    assert_worst(w)
+
+
+def test_one_sided_state_and_argument_errors():
+    from shampoo_second_order_b200 import Shampoo, _lib
+    opt = Shampoo([(64, 64), (32,)], 64, 0.9, 1e-6)
+    with pytest.raises(_lib.ShampooError) as e:
+        opt.set_one_sided(1, "left")                 # 1-D parameter
+    assert e.value.status == _lib.EINVAL
+    opt.set_one_sided(0, "left")
+    assert [opt.matrix_info(k)[1] for k in range(3)] == [2, 0, 2]
+    opt.set_one_sided(0, "both")
+    assert [opt.matrix_info(k)[1] for k in range(3)] == [4, 4, 2]
+    opt.update_stats([torch.randn(64, 64, device="cuda"), torch.randn(32, device="cuda")])
+    with pytest.raises(_lib.ShampooError) as e:
+        opt.set_one_sided(0, "right")                # after the first statistics
+    assert e.value.status == _lib.ESTATE
+    opt.close()
 
 
 # --------------------------------------------------------------------------
