@@ -59,26 +59,44 @@ def blocks_of(cfg):
     return blks, segs
 
 
+def block_sides(cfg):
+    """Per block, library order: 0 both factors, 2 R only (one-sided weights
+    listed in cfg["right_only"] by parameter index)."""
+    ro = set(cfg.get("right_only", ()))
+    out = []
+    b = cfg["block_size"]
+    for i, s in enumerate(cfg["shapes"]):
+        if len(s) == 2:
+            out += [2 if i in ro else 0] * (-(-s[0] // b) * -(-s[1] // b))
+    return out
+
+
 def matrix_sizes(cfg):
-    """(valid side, products per Newton step) per statistic, library order."""
+    """(valid side, products per Newton step) per statistic, library order;
+    a factor rooted at p/2 = 2 takes 3 products (X T, T T, T^2 M)."""
     blks, segs = blocks_of(cfg)
     out = []
-    for m, n in blks:
-        out += [(m, 4 if cfg["p"] == 4 else 3), (n, 4 if cfg["p"] == 4 else 3)]
+    for (m, n), sd in zip(blks, block_sides(cfg)):
+        pl = 4 if cfg["p"] == 4 and sd == 0 else 3
+        out += [(m, pl), (n, pl)]   # a dropped factor runs no iterations
     out += [(ln, 3 if cfg["p"] == 4 else 3) for ln in segs]   # p/2 = 2: X T, T T, T^2 M
     return out
 
 
 def stats_flops(cfg):
-    """SYRK triangles: m(m+1) n for L and n(n+1) m for R; len(len+1) per segment."""
+    """SYRK triangles: m(m+1) n for L and n(n+1) m for R (R only for a
+    one-sided block); len(len+1) per segment."""
     blks, segs = blocks_of(cfg)
-    return sum(m * (m + 1) * n + n * (n + 1) * m for m, n in blks) + sum(l * (l + 1) for l in segs)
+    return (sum((0 if sd else m * (m + 1) * n) + n * (n + 1) * m for (m, n), sd in zip(blks, block_sides(cfg)))
+            + sum(l * (l + 1) for l in segs))
 
 
 def apply_flops(cfg):
-    """Two chained GEMMs per block, 2mn(m+n); a matvec 2 len^2 per segment."""
+    """Two chained GEMMs per block, 2mn(m+n) (G R only, 2mn^2, for a one-sided
+    block); a matvec 2 len^2 per segment."""
     blks, segs = blocks_of(cfg)
-    return sum(2 * m * n * (m + n) for m, n in blks) + sum(2 * l * l for l in segs)
+    return (sum((2 * m * n * n if sd else 2 * m * n * (m + n)) for (m, n), sd in zip(blks, block_sides(cfg)))
+            + sum(2 * l * l for l in segs))
 
 
 def newton_flops(cfg, iters, per_kernel=False):
@@ -239,7 +257,8 @@ def tc_work(cfg, kernel):
     tri = T * (T + 1) // 2 * 128 * 128 * 4          # bytes of one statistic's upper tiles
     if kernel == "stats_tc":
         passes = 6 if f32 else 1
-        fl = sum(m * (m + 1) * n + n * (n + 1) * m for m, n in blks) * passes
+        fl = sum((0 if sd else m * (m + 1) * n) + n * (n + 1) * m
+                 for (m, n), sd in zip(blks, block_sides(cfg))) * passes
         by = sum(2 * planes * m * n for m, n in blks) + len(blks) * 2 * 2 * tri
     elif kernel == "apply_y_tc":
         passes = 3 if f32 else 2
@@ -479,6 +498,8 @@ def main():
     ap.add_argument("--roots", default="fp64", choices=["fp64", "int8"],
                     help="Newton products in float64 or emulated on the int8 tensor cores")
     ap.add_argument("--slices", type=int, default=6)
+    ap.add_argument("--one-sided-embedding", action="store_true",
+                    help="keep only R for embedding-like weights (rows >= 16 x cols)")
     args = ap.parse_args()
     if args.config == "batched_roots_512":
         return roots_bench(args)
@@ -532,6 +553,13 @@ def main():
     opt = Shampoo(shapes, cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"], cfg["graft"],
                   cfg["momentum"], cfg["grad_dtype"], stream=stream)
     opt.set_root_method(args.roots, args.slices)
+    one_sided = []
+    if args.one_sided_embedding:
+        for i, s_ in enumerate(shapes):
+            if len(s_) == 2 and s_[0] >= 16 * s_[1]:
+                opt.set_one_sided(i, "right")
+                one_sided.append(i)
+        cfg = dict(cfg, right_only=one_sided)   # the work model counts what is computed
     lr = cfg["lr"]
     interval = cfg["root_interval"]
 
@@ -707,6 +735,8 @@ def main():
                        "grad_dtype": cfg["grad_dtype"], "root_interval": interval,
                        "newton_products": (args.roots if args.roots == "fp64"
                                            else f"int8-emulated fp64, {args.slices} slices"),
+                       "one_sided_right": [list(shapes[i]) for i in one_sided],
+                       "one_sided_right": [list(shapes[i]) for i in one_sided],
                        "root_steps_timed": n_root, "l2": "flushed between steps (256 MiB write)",
                        "parallelism": f"replicas x{world}"},
             "roofline": roof, "cpu_baseline": cpu_line, "e2e": e2e, "async_roots": async_line,
