@@ -482,6 +482,81 @@ def roots_bench(args):
 # ---------------------------------------------------------------------------
 # the CUDA arm
 # ---------------------------------------------------------------------------
+def shard_bench(args, cfg, rank, world, local):
+    """Block-sharded data parallelism: one parameter set, each rank owning a
+    share of the parameters (shampoo_plan_shards), gradients reduce-scattered
+    to their owners and updated weights all-gathered, every step inside the
+    timed region.  value = the whole set's work / the slowest rank's time."""
+    import torch
+    import torch.distributed as dist
+    from shampoo_second_order_b200.sharded import ShardedShampoo
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    stream = torch.cuda.Stream(device=dev, priority=-1)
+    shapes = cfg["shapes"]
+    gdt = torch.bfloat16 if cfg["grad_dtype"] == "bf16" else torch.float32
+    interval = cfg["root_interval"]
+    W0 = wl.make_params(shapes, cfg["seed"])
+    NG = 2
+    with torch.cuda.stream(stream):
+        W = [torch.from_numpy(w).to(dev) for w in W0]
+        G = [[torch.from_numpy(g).to(dev).to(gdt)
+              for g in wl.make_grads(shapes, cfg["seed"] + 17 * rank, t, cfg["grad_std"], cfg["grad_dtype"])]
+             for t in range(NG)]
+        flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    stream.synchronize()
+    opt = ShardedShampoo(shapes, cfg["block_size"], cfg["beta2"], cfg["eps"], cfg["p"], cfg["graft"],
+                         cfg["momentum"], cfg["grad_dtype"], interval, stream=stream)
+    with torch.cuda.stream(stream):
+        for t in range(args.warmup):
+            opt.step(W, G[t % NG], cfg["lr"], t == 0)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    iters = None
+    with torch.cuda.stream(stream):
+        for j in range(args.steps):
+            flush.zero_()
+            ev[j][0].record(stream)
+            roots = j % interval == 0
+            opt.step(W, G[j % NG], cfg["lr"], roots)
+            ev[j][1].record(stream)
+            if roots and opt.local is not None:
+                its = opt.local.root_iterations()
+                iters = its if iters is None else [a + b for a, b in zip(iters, its)]
+    stream.synchronize()
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), dist if world > 1 else None, dev)
+    sub = dict(cfg, shapes=[shapes[i] for i in opt.mine])
+    newton = newton_flops(sub, iters) if iters else 0
+    if world > 1:
+        t = torch.tensor([float(newton)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t)
+        newton = float(t.item())
+    flops = args.steps * (stats_flops(cfg) + apply_flops(cfg)) + newton
+    if rank == 0:
+        line = {"metric": METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32/f64",
+                "data": "synthetic",
+                "config": {"workload": args.config, "params": numel(cfg), "block_size": cfg["block_size"],
+                           "grad_dtype": cfg["grad_dtype"], "root_interval": interval,
+                           "parallelism": f"block-sharded dp{world}",
+                           "collective_bytes_per_rank_step": opt.collective_bytes_per_step(),
+                           "planned_cost_balance": round(min(opt.planned_cost) / max(opt.planned_cost), 4),
+                           "l2": "flushed between steps (256 MiB write)"}}
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -498,6 +573,9 @@ def main():
     ap.add_argument("--roots", default="fp64", choices=["fp64", "int8"],
                     help="Newton products in float64 or emulated on the int8 tensor cores")
     ap.add_argument("--slices", type=int, default=6)
+    ap.add_argument("--shard", action="store_true",
+                    help="one parameter set split over the ranks by owner (strong scaling, with the "
+                         "gradient reduce-scatter and weight all-gather)")
     ap.add_argument("--one-sided-embedding", action="store_true",
                     help="keep only R for embedding-like weights (rows >= 16 x cols)")
     args = ap.parse_args()
@@ -512,6 +590,8 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, cfg, rank, world)
+    if args.shard:
+        return shard_bench(args, cfg, rank, world, local)
 
     # CPU baseline first (rank 0, N = 1 only), before any GPU work
     cpu = None

@@ -373,6 +373,31 @@ shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, float* X, in
                                                     int p, float eps, double tol, int max_iters,
                                                     int32_t* iters, void* stream);
 
+/*
+ * shampoo_plan_shards -- which rank owns each parameter in the block-sharded
+ * data-parallel step.  The blocks of a weight are independent (podcast
+ * transcript, segment 16, Lemma 2), so ranks split the optimizer work by
+ * whole parameter: each owner receives the summed gradients of its
+ * parameters, runs statistics, roots and apply on them alone (the
+ * layer-wise graft stays local) and sends the updated weights to the others.
+ *  nparams, shapes, ndims, block_size  as for shampoo_create (host arrays).
+ *  root_interval  steps between root computations (>= 1), to weigh the
+ *                 root work against the per-step work.
+ *  nranks   >= 1.
+ *  owner    host int32 [nparams] output: the owning rank of each parameter.
+ *  rank_cost  host double [nranks] output or NULL: the planned work per
+ *             rank, in the planner's flop-like units.
+ * Longest-processing-time-first over a per-parameter cost model (statistics
+ * and apply GEMMs per step, root products per root interval, elementwise
+ * passes); deterministic, so every rank computes the same plan.  Host only:
+ * touches no GPU.  SHAMPOO_EINVAL on bad arguments (message from
+ * shampoo_last_error(NULL)).
+ */
+shampoo_status shampoo_plan_shards(int nparams, const int64_t* shapes,
+                                   const int32_t* ndims, int block_size,
+                                   int root_interval, int nranks, int32_t* owner,
+                                   double* rank_cost);
+
 /* Library version, "MAJOR.MINOR.PATCH". */
 const char* shampoo_version(void);
 

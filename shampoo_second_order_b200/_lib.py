@@ -50,6 +50,8 @@ SIGNATURES = {
                                                   C.c_double, C.c_int, _P, _P, C.c_int, C.c_int]),
     "shampoo_batched_inverse_root_noalloc": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_float,
                                                        C.c_double, C.c_int, _P, _P]),
+    "shampoo_plan_shards": (C.c_int, [C.c_int, C.POINTER(C.c_int64), C.POINTER(C.c_int32), C.c_int, C.c_int,
+                                      C.c_int, C.POINTER(C.c_int32), C.POINTER(C.c_double)]),
     "shampoo_version": (C.c_char_p, []),
 }
 
@@ -229,6 +231,22 @@ def shampoo_batched_inverse_root_noalloc(A_ptr, X_ptr, batch, n, p, eps, tol, ma
                                                     int(max_iters), C.c_void_p(int(iters_ptr)),
                                                     C.c_void_p(int(stream)))
     return _check(st, None, allow=(ENOTCONVERGED,))
+
+
+def shampoo_plan_shards(shapes, block_size, root_interval, nranks):
+    """(owner per parameter, planned cost per rank); host only."""
+    n = len(shapes)
+    dims = (C.c_int64 * (2 * n))()
+    nd = (C.c_int32 * n)()
+    for i, s in enumerate(shapes):
+        if len(s) == 1:
+            dims[2 * i], dims[2 * i + 1], nd[i] = 1, int(s[0]), 1
+        else:
+            dims[2 * i], dims[2 * i + 1], nd[i] = int(s[0]), int(s[1]), 2
+    owner = (C.c_int32 * n)()
+    cost = (C.c_double * int(nranks))()
+    _check(lib().shampoo_plan_shards(n, dims, nd, int(block_size), int(root_interval), int(nranks), owner, cost))
+    return list(owner), list(cost)
 
 
 def shampoo_version():

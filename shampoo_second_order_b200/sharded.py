@@ -1,0 +1,112 @@
+"""Block-sharded data-parallel Shampoo over torch.distributed.
+
+The blocks of a weight are independent (podcast transcript, segment 16,
+Lemma 2), so data-parallel ranks split the optimizer work by whole
+parameter.  Every rank computes the gradients of all parameters on its own
+data; each step then
+
+  1. reduce-scatters the gradients: one collective over a buffer laid out by
+     owner leaves on each rank the sum, over ranks, of the gradients of the
+     parameters it owns, scaled by 1/world (the data-parallel mean);
+  2. runs update_stats, compute_roots (when due) and apply for its own
+     parameters through its own library context -- a parameter's blocks and
+     its layer-wise graft norms never leave its owner;
+  3. all-gathers the updated weights, so every rank holds the whole model.
+
+Collective bytes per rank and step: the gradient buffer (world x the largest
+owner share, in the gradient dtype) and the weight buffer (the same, float32).
+Ownership comes from shampoo_plan_shards, which every rank evaluates to the
+same plan.  With one process (no process group) the collectives are skipped.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import _lib as L
+
+_ALIGN = 16   # elements: every parameter's slice of a flat buffer starts 64-byte aligned
+
+
+class ShardedShampoo:
+    """shapes, block_size, beta2, eps, p, graft, momentum, grad_dtype: as for
+    Shampoo.  root_interval: steps between root computations (weighs the
+    plan).  group: a torch.distributed process group (default: the world).
+    make_local(shapes) builds the per-rank optimizer over the owned shapes;
+    the default is a Shampoo context on the current CUDA device and stream.
+    """
+
+    def __init__(self, shapes, block_size, beta2, eps, p=4, graft=L.GRAFT_ADAGRAD, momentum=0.0,
+                 grad_dtype="f32", root_interval=1, group=None, make_local=None, stream=None):
+        import torch
+        import torch.distributed as dist
+        self._dist = dist
+        self.shapes = [tuple(int(d) for d in s) for s in shapes]
+        self.group = group
+        on = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size(group) if on else 1
+        self.rank = dist.get_rank(group) if on else 0
+        self.owner, self.planned_cost = L.shampoo_plan_shards(self.shapes, block_size, root_interval, self.world)
+        self.numel = [int(np.prod(s)) for s in self.shapes]
+        self.off = [0] * len(self.shapes)
+        size = [0] * self.world
+        for i, o in enumerate(self.owner):
+            self.off[i] = size[o]
+            size[o] += -(-self.numel[i] // _ALIGN) * _ALIGN
+        self.pad = max(max(size), _ALIGN)
+        self.mine = [i for i, o in enumerate(self.owner) if o == self.rank]
+        if make_local is None:
+            from .optimizer import Shampoo
+
+            def make_local(sh):
+                return Shampoo(sh, block_size, beta2, eps, p, graft, momentum, grad_dtype, stream)
+        self.local = make_local([self.shapes[i] for i in self.mine]) if self.mine else None
+        self.gdtype = torch.bfloat16 if grad_dtype == "bf16" else torch.float32
+        self._bufs = None
+
+    def collective_bytes_per_step(self):
+        g = 2 if self.gdtype.itemsize == 2 else 4
+        return self.world * self.pad * (g + 4)
+
+    def _buffers(self, device):
+        import torch
+        if self._bufs is None:
+            n = self.world * self.pad
+            self._bufs = (torch.zeros(n, dtype=self.gdtype, device=device),        # gradients by owner
+                          torch.zeros(self.pad, dtype=self.gdtype, device=device),  # this rank's summed share
+                          torch.zeros(self.pad, dtype=torch.float32, device=device),
+                          torch.zeros(n, dtype=torch.float32, device=device))
+        return self._bufs
+
+    def step(self, params, grads, lr, compute_roots):
+        """params: all parameters (float32, updated in place on every rank);
+        grads: this rank's gradients of all parameters."""
+        dist = self._dist
+        send, recv, wmine, wall = self._buffers(params[0].device)
+        for i, g in enumerate(grads):
+            o = self.owner[i] * self.pad + self.off[i]
+            send[o:o + self.numel[i]].copy_(g.reshape(-1))
+        if self.world > 1:
+            dist.reduce_scatter_tensor(recv, send, group=self.group)
+            recv.mul_(1.0 / self.world)
+        else:
+            recv.copy_(send[:self.pad])
+        if self.local is not None:
+            gm = [recv[self.off[i]:self.off[i] + self.numel[i]].view(self.shapes[i]) for i in self.mine]
+            pm = [params[i] for i in self.mine]
+            self.local.update_stats(gm)
+            if compute_roots:
+                self.local.compute_roots()
+            self.local.apply(pm, gm, lr)
+        if self.world > 1:
+            for i in self.mine:
+                wmine[self.off[i]:self.off[i] + self.numel[i]].copy_(params[i].reshape(-1))
+            dist.all_gather_into_tensor(wall, wmine, group=self.group)
+            for i, o in enumerate(self.owner):
+                if o != self.rank:
+                    a = o * self.pad + self.off[i]
+                    params[i].copy_(wall[a:a + self.numel[i]].view(self.shapes[i]))
+
+    def close(self):
+        if self.local is not None and hasattr(self.local, "close"):
+            self.local.close()
+        self.local = None
