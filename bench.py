@@ -39,7 +39,12 @@ UNIT = "TFLOP/s"
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
 # ncu capture of the named kernel; None until measured for the current kernel.
-TRAFFIC_PER_LAUNCH = {}
+TRAFFIC_PER_LAUNCH = {
+    # the 9 launches of the timed root step of the default Transformer-layer
+    # run (5 with every matrix iterating: ~1.01 GB each; 3 with a few: 17 MB;
+    # 1 with none), averaged like `achieved`
+    "newton_step_a": 565950948,
+}
 
 
 # ---------------------------------------------------------------------------
