@@ -304,7 +304,7 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
       for (const auto& m : list) has_p4 |= (m.p == 4);
       run(pr, "newton_reset", st, [&] { launch_newton_reset(nm, w, st); });
       run(pr, "newton_bound", st, [&] {
-        launch_newton_bound(A, a_stride, lda, upper, d, nm, eps, attempt, w, st);
+        launch_newton_bound(A, a_stride, lda, upper, d, nm, S, eps, attempt, w, st);
       });
       run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, upper, d, nm, S, w, st); });
       run(pr, "newton_lanczos", st, [&] { launch_newton_lanczos(d, nm, S, w, st); });

@@ -128,7 +128,7 @@ void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s);
 // upper: A holds only its upper-triangular 128 x 128 tiles; element (r, c)
 // of a lower tile is read from (c, r).
 void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
-                         int nm, float eps, int attempt, NewtonWork w, cudaStream_t s);
+                         int nm, int S, float eps, int attempt, NewtonWork w, cudaStream_t s);
 void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
                         int nm, int S, NewtonWork w, cudaStream_t s);
 // Lanczos estimate of M0's spectrum and the scaling schedule, then T0.

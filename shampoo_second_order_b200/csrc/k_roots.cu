@@ -164,44 +164,89 @@ __device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0,
 // ---------------------------------------------------------------------------
 // Set-up: the eigenvalue bound, X0, M0, T0 and the first residual.
 // ---------------------------------------------------------------------------
-// One CTA per matrix: c^p = min(||A + eps I||_F, ||A + eps I||_inf) over the
-// valid corner.  Both bound the largest eigenvalue of a symmetric matrix.
-// On a retry (attempt k > 0) the ridge is raised to eps + 8^k 2^-24 c^p:
-// rounding of a float32 statistic can leave eigenvalues of A + eps I below
-// zero by about 2^-24 c^p, which the iteration cannot root.
+// Element (r, c) of a statistic stored as upper 128-tiles (upper = 1) or in
+// full (upper = 0).
 __device__ __forceinline__ float sym_at(const float* a, int lda, int upper, int r, int c) {
   if (upper && (r >> 7) > (c >> 7)) return a[(size_t)c * lda + r];
   return a[(size_t)r * lda + c];
 }
 
-__global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restrict__ A,
-                                                           int64_t a_stride, int lda, int upper,
-                                                           const NewtonMat* __restrict__ mats,
-                                                           float eps, int attempt,
-                                                           double* __restrict__ cinv,
-                                                           double* __restrict__ ridge,
-                                                           double* __restrict__ cpow) {
+// grid: x = band of 32 rows, y = matrix.  Partial sums of the bound over the
+// valid corner: ||A + eps I||_F^2 into fro2[m] and the absolute row sums into
+// rows[m][:].  A statistic stored as upper 128-tiles is read row by row: an
+// entry of an off-diagonal tile stands for itself and its mirror, so it adds
+// twice to the Frobenius sum and to the row sums of both its row and its
+// column (the column part accumulated per lane, then per block in shared
+// memory, then once per block in global memory).
+__global__ void __launch_bounds__(256) newton_bound_partial_kernel(const float* __restrict__ A,
+                                                                   int64_t a_stride, int lda, int upper,
+                                                                   const NewtonMat* __restrict__ mats,
+                                                                   int S, float eps,
+                                                                   double* __restrict__ fro2,
+                                                                   double* __restrict__ rows) {
   __shared__ double red[8];
-  const NewtonMat mt = mats[blockIdx.x];
+  __shared__ double colsum[1024];
+  const int m = blockIdx.y;
+  const NewtonMat mt = mats[m];
   const float* a = A + (size_t)mt.slot * a_stride;
   const int n = mt.size;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double fro = 0.0, rowmax = 0.0;
-  for (int r = warp; r < n; r += 8) {
+  for (int c = threadIdx.x; c < S; c += blockDim.x) colsum[c] = 0.0;
+  __syncthreads();
+  double* rsum = rows + (size_t)m * S;
+  double fro = 0.0;
+  double col[32];   // this lane's mirror contributions, columns lane + 32 k
+#pragma unroll
+  for (int k = 0; k < 32; ++k) col[k] = 0.0;
+  for (int j = 0; j < 4; ++j) {
+    const int r = blockIdx.x * 32 + warp + 8 * j;
+    if (r >= n) continue;
+    const float* row = a + (size_t)r * lda;
     double rs = 0.0;
-    for (int c = lane; c < n; c += 32) {
-      double v = (double)sym_at(a, lda, upper, r, c);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= n) continue;
+      const bool mirror = upper && (c >> 7) > (r >> 7);
+      if (upper && (c >> 7) < (r >> 7)) continue;   // a lower tile: never written
+      double v = (double)row[c];
       if (r == c) v += (double)eps;
       rs += fabs(v);
-      fro += v * v;
+      fro += (mirror ? 2.0 : 1.0) * v * v;
+      if (mirror) col[k] += fabs(v);
     }
     rs = warp_sum(rs);
-    rowmax = fmax(rowmax, rs);
+    if (lane == 0 && rs != 0.0) atomicAdd(&rsum[r], rs);
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int c = lane + 32 * k;
+    if (c < n && col[k] != 0.0) atomicAdd(&colsum[c], col[k]);
   }
   fro = block_sum(fro, red);
-  rowmax = block_max(rowmax, red);
-  if (threadIdx.x == 0) {
-    double cp = fmin(sqrt(fro), rowmax);
+  __syncthreads();
+  for (int c = threadIdx.x; c < n; c += blockDim.x)
+    if (colsum[c] != 0.0) atomicAdd(&rsum[c], colsum[c]);
+  if (threadIdx.x == 0 && fro != 0.0) atomicAdd(&fro2[m], fro);
+}
+
+// One warp per matrix: c^p = min(||A + eps I||_F, ||A + eps I||_inf), both
+// bounds of the largest eigenvalue of a symmetric matrix, from the partial
+// sums; then the residual and Frobenius slots are cleared for the iteration.
+// On a retry (attempt k > 0) the ridge is raised to eps + 8^k 2^-24 c^p:
+// rounding of a float32 statistic can leave eigenvalues of A + eps I below
+// zero by about 2^-24 c^p, which the iteration cannot root.
+__global__ void newton_bound_final_kernel(const NewtonMat* __restrict__ mats, int nm, int S, float eps,
+                                          int attempt, NewtonWork w, const double* __restrict__ rows,
+                                          double* __restrict__ cpow) {
+  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (m >= nm) return;
+  const NewtonMat mt = mats[m];
+  double rowmax = 0.0;
+  for (int c = lane; c < mt.size; c += 32) rowmax = fmax(rowmax, rows[(size_t)m * S + c]);
+  rowmax = warp_max(rowmax);
+  if (lane == 0) {
+    double cp = fmin(sqrt(w.fro2[m]), rowmax);
     if (!(cp > 0.0) || !(cp <= DBL_MAX)) cp = (cp > 0.0) ? cp : 1.0;  // NaN/Inf/0 caught later
     double rd = (double)eps;
     if (attempt > 0) {
@@ -209,9 +254,11 @@ __global__ void __launch_bounds__(256) newton_bound_kernel(const float* __restri
       rd += extra;
       cp += extra;   // lambda_max grows by exactly the added ridge
     }
-    ridge[blockIdx.x] = rd;
-    cpow[blockIdx.x] = cp;
-    cinv[blockIdx.x] = pow(cp, -1.0 / mt.p);
+    w.ridge[m] = rd;
+    cpow[m] = cp;
+    w.cinv[m] = pow(cp, -1.0 / mt.p);
+    w.fro2[m] = 0.0;
+    w.resid[m] = 0ull;
   }
 }
 
@@ -617,12 +664,14 @@ void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s) {
   newton_reset_kernel<<<1, 1024, 0, s>>>(nm, w);
 }
 
-// c^p goes to the first nm doubles of T2, which no step reads before step A
-// overwrites it.
+// c^p goes to the first nm doubles of T2, and the row sums to the first
+// nm * S doubles of T: no step reads either before step A / T0 overwrite them.
 void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
-                         int nm, float eps, int attempt, NewtonWork w, cudaStream_t s) {
-  newton_bound_kernel<<<nm, 256, 0, s>>>(A, a_stride, lda, upper, mats, eps, attempt, w.cinv,
-                                         w.ridge, w.T2);
+                         int nm, int S, float eps, int attempt, NewtonWork w, cudaStream_t s) {
+  cudaMemsetAsync(w.T, 0, (size_t)nm * S * sizeof(double), s);
+  newton_bound_partial_kernel<<<dim3((S + 31) / 32, nm), 256, 0, s>>>(A, a_stride, lda, upper, mats, S, eps,
+                                                                      w.fro2, w.T);
+  newton_bound_final_kernel<<<(nm + 7) / 8, 256, 0, s>>>(mats, nm, S, eps, attempt, w, w.T, w.T2);
 }
 
 void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,

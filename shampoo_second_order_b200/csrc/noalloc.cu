@@ -188,7 +188,7 @@ extern "C" shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, f
     fill_mats_kernel<<<(nm + 127) / 128, 128, 0, st>>>(mats, nm, c0, n, p);
     for (int attempt = 0; attempt < kAttemptsNoAlloc && nm > 0 && e == cudaSuccess; ++attempt) {
       launch_newton_reset(nm, w, st);
-      launch_newton_bound(A, (int64_t)n * n, n, 0, mats, nm, eps, attempt, w, st);
+      launch_newton_bound(A, (int64_t)n * n, n, 0, mats, nm, S, eps, attempt, w, st);
       launch_newton_init(A, (int64_t)n * n, n, 0, mats, nm, S, w, st);
       launch_newton_lanczos(mats, nm, S, w, st);
       launch_newton_t0(mats, nm, S, w, st);
