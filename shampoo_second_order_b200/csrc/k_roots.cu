@@ -377,18 +377,55 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
   double beta = 0.0;
   int kk = 0;
   for (int j = 0; j < kLanczos && j < n; ++j) {
-    for (int r = warp; r < n; r += nw) {
-      // 16-byte loads; column n of an odd-sized corner is padding (0 here)
-      const double2* row = reinterpret_cast<const double2*>(M + (size_t)r * S);
-      double d0 = 0.0, d1 = 0.0;
-#pragma unroll 4
-      for (int c2 = lane; c2 < n2; c2 += 32) {
-        const double2 x = row[c2];
-        d0 = fma(x.x, v[2 * c2], d0);
-        d1 = fma(x.y, v[2 * c2 + 1], d1);
+    // the matvec streams M0 from memory: every 16-byte load of a warp's rows
+    // is issued before the first is used, so the loads of a row are in flight
+    // together (two rows per warp while n <= 512)
+    if (n2 <= 256) {
+      for (int r = 2 * warp; r < n; r += 2 * nw) {
+        const bool two = r + 1 < n;
+        const double2* row0 = reinterpret_cast<const double2*>(M + (size_t)r * S);
+        const double2* row1 = reinterpret_cast<const double2*>(M + (size_t)(two ? r + 1 : r) * S);
+        double2 x0[8], x1[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c2 = lane + 32 * k;
+          x0[k] = c2 < n2 ? row0[c2] : make_double2(0.0, 0.0);
+          x1[k] = c2 < n2 ? row1[c2] : make_double2(0.0, 0.0);
+        }
+        double d0 = 0.0, d1 = 0.0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c2 = lane + 32 * k;
+          if (c2 < n2) {
+            d0 = fma(x0[k].x, v[2 * c2], fma(x0[k].y, v[2 * c2 + 1], d0));
+            d1 = fma(x1[k].x, v[2 * c2], fma(x1[k].y, v[2 * c2 + 1], d1));
+          }
+        }
+        d0 = warp_sum(d0);
+        d1 = warp_sum(d1);
+        if (lane == 0) {
+          wv[r] = d0 - beta * vp[r];
+          if (two) wv[r + 1] = d1 - beta * vp[r + 1];
+        }
       }
-      const double d = warp_sum(d0 + d1);
-      if (lane == 0) wv[r] = d - beta * vp[r];
+    } else {
+      for (int r = warp; r < n; r += nw) {
+        const double2* row = reinterpret_cast<const double2*>(M + (size_t)r * S);
+        double2 x[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int c2 = lane + 32 * k;
+          x[k] = c2 < n2 ? row[c2] : make_double2(0.0, 0.0);
+        }
+        double d = 0.0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int c2 = lane + 32 * k;
+          if (c2 < n2) d = fma(x[k].x, v[2 * c2], fma(x[k].y, v[2 * c2 + 1], d));
+        }
+        d = warp_sum(d);
+        if (lane == 0) wv[r] = d - beta * vp[r];
+      }
     }
     __syncthreads();
     double a = 0.0;
