@@ -264,6 +264,9 @@ __global__ void newton_bound_final_kernel(const NewtonMat* __restrict__ mats, in
 
 // grid: x = row of the S x S slot, y = matrix.  Writes X0, M0 into the
 // parity-0 buffers and folds max|M0 - I| (valid corner) into the residual.
+// Also writes the valid corner of the statistic itself, mirrored, as float32
+// into T4 (unused until the first step B): the Lanczos run multiplies by it,
+// which is M0 up to the ridge and the scale c^p, at half the bytes.
 __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restrict__ A,
                                                           int64_t a_stride, int lda, int upper,
                                                           const NewtonMat* __restrict__ mats,
@@ -279,6 +282,7 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
   const double rd = w.ridge[m];
   const double ci = w.cinv[m];
   double dev = 0.0;
+  float* a32 = reinterpret_cast<float*>(w.T4 + (size_t)m * S * S) + (size_t)r * S;
   for (int c = threadIdx.x; c < S; c += blockDim.x) {
     double v;
     const bool valid = r < mt.size && c < mt.size;
@@ -286,10 +290,12 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
       // a full input is read through its symmetric part (exact when symmetric)
       v = upper ? (double)sym_at(a, lda, upper, r, c)
                 : 0.5 * ((double)a[(size_t)r * lda + c] + (double)a[(size_t)c * lda + r]);
+      a32[c] = (float)v;
       if (r == c) v += rd;
       v *= inv_cp;
     } else {
       v = (r == c) ? 1.0 : 0.0;
+      a32[c] = 0.f;
     }
     const double d = (r == c) ? 1.0 : 0.0;
     w.M[0][off + c] = v;
@@ -343,7 +349,8 @@ __device__ double tridiag_eig(const double* a, const double* b, int k, int which
 }
 
 // One CTA per matrix: kLanczos Lanczos steps on the valid corner of M0
-// (float64, no reorthogonalisation: only the extreme Ritz values are used),
+// (float64 vectors, the float32 statistic as the operator; no
+// reorthogonalisation: only the extreme Ritz values are used),
 // their extreme eigenvalues by Sturm bisection, and the schedule s_k.
 __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __restrict__ mats, int S,
                                                              NewtonWork w) {
@@ -354,7 +361,8 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
   const int m = blockIdx.x;
   const NewtonMat mt = mats[m];
   const int n = mt.size, p = mt.p;
-  const double* M = w.M[0] + (size_t)m * S * S;
+  const float* A32 = reinterpret_cast<const float*>(w.T4 + (size_t)m * S * S);   // written by newton_init
+  const double rd = w.ridge[m], inv_cp = 1.0 / w.T2[m];                       // T2 holds c^p until step A
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   // start vector: a fixed pseudo-random +-1 pattern (hash of the index)
   double ss = 0.0;
@@ -371,60 +379,45 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
   __syncthreads();
   const double inv0 = bcast;
   for (int i = threadIdx.x; i < n; i += blockDim.x) v[i] *= inv0;
-  if (threadIdx.x == 0 && (n & 1)) v[n] = 0.0;   // pad for the pairwise row loads
+  const int n4 = (n + 3) >> 2;
+  if (threadIdx.x < 4 * n4 - n) v[n + threadIdx.x] = 0.0;   // pad for the 4-wide row loads
   __syncthreads();
-  const int n2 = (n + 1) >> 1;
   double beta = 0.0;
   int kk = 0;
   for (int j = 0; j < kLanczos && j < n; ++j) {
-    // the matvec streams M0 from memory: every 16-byte load of a warp's rows
-    // is issued before the first is used, so the loads of a row are in flight
-    // together (two rows per warp while n <= 512)
-    if (n2 <= 256) {
-      for (int r = 2 * warp; r < n; r += 2 * nw) {
-        const bool two = r + 1 < n;
-        const double2* row0 = reinterpret_cast<const double2*>(M + (size_t)r * S);
-        const double2* row1 = reinterpret_cast<const double2*>(M + (size_t)(two ? r + 1 : r) * S);
-        double2 x0[8], x1[8];
+    // M0 v = ((A + ridge I) v) / c^p with A the float32 statistic (exact
+    // values) streamed from memory; every 16-byte load of a warp's two rows is
+    // issued before the first is used
+    for (int r = 2 * warp; r < n; r += 2 * nw) {
+      const bool two = r + 1 < n;
+      const float4* row0 = reinterpret_cast<const float4*>(A32 + (size_t)r * S);
+      const float4* row1 = reinterpret_cast<const float4*>(A32 + (size_t)(two ? r + 1 : r) * S);
+      double d0 = 0.0, d1 = 0.0;
+      for (int base = 0; base < n4; base += 128) {   // 512 columns at a time
+        float4 x0[4], x1[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int c2 = lane + 32 * k;
-          x0[k] = c2 < n2 ? row0[c2] : make_double2(0.0, 0.0);
-          x1[k] = c2 < n2 ? row1[c2] : make_double2(0.0, 0.0);
+        for (int k = 0; k < 4; ++k) {
+          const int c4 = base + lane + 32 * k;
+          x0[k] = c4 < n4 ? row0[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          x1[k] = c4 < n4 ? row1[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        double d0 = 0.0, d1 = 0.0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int c2 = lane + 32 * k;
-          if (c2 < n2) {
-            d0 = fma(x0[k].x, v[2 * c2], fma(x0[k].y, v[2 * c2 + 1], d0));
-            d1 = fma(x1[k].x, v[2 * c2], fma(x1[k].y, v[2 * c2 + 1], d1));
+        for (int k = 0; k < 4; ++k) {
+          const int c4 = base + lane + 32 * k;
+          if (c4 < n4) {
+            const int c = 4 * c4;
+            d0 = fma((double)x0[k].x, v[c], fma((double)x0[k].y, v[c + 1],
+                     fma((double)x0[k].z, v[c + 2], fma((double)x0[k].w, v[c + 3], d0))));
+            d1 = fma((double)x1[k].x, v[c], fma((double)x1[k].y, v[c + 1],
+                     fma((double)x1[k].z, v[c + 2], fma((double)x1[k].w, v[c + 3], d1))));
           }
         }
-        d0 = warp_sum(d0);
-        d1 = warp_sum(d1);
-        if (lane == 0) {
-          wv[r] = d0 - beta * vp[r];
-          if (two) wv[r + 1] = d1 - beta * vp[r + 1];
-        }
       }
-    } else {
-      for (int r = warp; r < n; r += nw) {
-        const double2* row = reinterpret_cast<const double2*>(M + (size_t)r * S);
-        double2 x[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int c2 = lane + 32 * k;
-          x[k] = c2 < n2 ? row[c2] : make_double2(0.0, 0.0);
-        }
-        double d = 0.0;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int c2 = lane + 32 * k;
-          if (c2 < n2) d = fma(x[k].x, v[2 * c2], fma(x[k].y, v[2 * c2 + 1], d));
-        }
-        d = warp_sum(d);
-        if (lane == 0) wv[r] = d - beta * vp[r];
+      d0 = warp_sum(d0);
+      d1 = warp_sum(d1);
+      if (lane == 0) {
+        wv[r] = (d0 + rd * v[r]) * inv_cp - beta * vp[r];
+        if (two) wv[r + 1] = (d1 + rd * v[r + 1]) * inv_cp - beta * vp[r + 1];
       }
     }
     __syncthreads();
@@ -454,7 +447,7 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
       vp[i] = v[i];
       v[i] = wv[i] / b;
     }
-    beta = b;   // v[n] stays 0 for odd n
+    beta = b;   // the padding v[n .. 4 n4) stays 0
     __syncthreads();
   }
   __syncthreads();
