@@ -317,6 +317,7 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
       run(pr, "newton_check", st, [&] { launch_newton_check(nm, 0, tol, max_iters, w, st); });
       CK(cudaMemcpyAsync(&h_count[0], &w.count[0], sizeof(int), cudaMemcpyDeviceToHost, st));
       CK(cudaEventRecord(ev[0], st));
+      int known = nm;   // matrices iterating, as last read back (an upper bound)
       for (int it = 0; it < max_iters; ++it) {
         // the check of M_it is in flight; queue step it+1 before waiting for it
         if (oz) {   // the same step with emulated float64 products on the int8 tensor cores
@@ -334,9 +335,14 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
           });
           if (oe != cudaSuccess) return cuda_fail(ctx, oe, "emulated Newton step");
         } else {
-          run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, w, st); });
-          if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, w, st); });
-          run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, w, st); });
+          // 32 x 32 tiles once so few matrices are left (the count known on
+          // the host bounds the running ones) that 64 x 64 tiles would fill
+          // under two CTAs per SM
+          const int t64 = (S / 64) * (S / 64 + 1) / 2;
+          const int tile = (int64_t)known * t64 * 2 <= 2 * 148 ? 32 : 64;
+          run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, tile, w, st); });
+          if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, tile, w, st); });
+          run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, tile, w, st); });
         }
         run(pr, "newton_check", st, [&] { launch_newton_check(nm, it + 1, tol, max_iters, w, st); });
         const int nx = (it + 1) & 1;
@@ -345,6 +351,7 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
         CK(cudaEventRecord(ev[nx], st));
         CK(cudaEventSynchronize(ev[it & 1]));
         if (h_count[it & 1] == 0) break;
+        known = h_count[it & 1];
       }
       CK(cudaMemcpyAsync(hstate.data(), w.state, nm * sizeof(int), cudaMemcpyDeviceToHost, st));
       CK(cudaMemcpyAsync(hiters.data(), w.iters, nm * sizeof(int), cudaMemcpyDeviceToHost, st));

@@ -135,10 +135,11 @@ void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, co
 void launch_newton_lanczos(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
 void launch_newton_t0(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
 // one Newton step: A (X T and T T), B (T2 T2, p = 4 only), C (T^p M,
-// residual, next T); check k: convergence test of M_k
-void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);
-void launch_newton_step_b(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s);
-void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s);
+// residual, next T) on tiles of side `tile` (64, or 32 when few matrices are
+// left); check k: convergence test of M_k
+void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s);
+void launch_newton_step_b(const NewtonMat* mats, int nm, int S, int tile, NewtonWork w, cudaStream_t s);
+void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s);
 void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s);
 
 // ---------------- emulated float64 Newton products (k_ozaki.cu) ----------------

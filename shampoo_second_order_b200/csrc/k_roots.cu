@@ -40,7 +40,6 @@ namespace {
 constexpr int kNewtonThreads = 128;
 constexpr int kBK = 16;
 constexpr int kAStride = kBK + 4;     // doubles; 4 mod 16 keeps fragment loads conflict-free
-constexpr int kBStride = kTile + 4;
 
 enum : int { kRunning = 0, kConverged = 1, kFailed = 2, kDiverged = 3, kFinal = 4 };
 
@@ -73,35 +72,40 @@ __device__ __forceinline__ void tri_tile(int idx, int T, int& ti, int& tj) {
   tj = ti + idx;
 }
 
+// Tile side TT (64, or 32 for the last steps, when only a few matrices are
+// left and 64 x 64 tiles would leave most SMs idle).
+template <int TT>
 struct NewtonSmem {
-  double As[2][kTile][kAStride];
-  double Bs[2][kBK][kBStride];
+  double As[2][TT][kAStride];
+  double Bs[2][kBK][TT + 4];   // row stride = 8 mod 32 words: conflict-free fragment loads
 };
 
-// acc = A[i0:i0+64, :] * B[:, j0:j0+64] for S x S row-major float64 A, B.
-// 4 warps in a 2 x 2 arrangement, each a 32 x 32 sub-tile of 4 x 4 m8n8
-// fragments; lane (g, t) = (lane / 4, lane % 4) holds acc[mi][ni][e] at row
-// 8 mi + g, column 8 ni + 2 t + e of its sub-tile.
+// acc = A[i0:i0+TT, :] * B[:, j0:j0+TT] for S x S row-major float64 A, B.
+// 4 warps in a 2 x 2 arrangement, each a TT/2 x TT/2 sub-tile of FM x FM
+// m8n8 fragments (FM = TT/16); lane (g, t) = (lane / 4, lane % 4) holds
+// acc[mi][ni][e] at row 8 mi + g, column 8 ni + 2 t + e of its sub-tile.
+template <int TT>
 __device__ __forceinline__ void dmma_tile(const double* __restrict__ A, const double* __restrict__ B,
-                                          int S, int i0, int j0, double acc[4][4][2],
-                                          NewtonSmem& sm) {
+                                          int S, int i0, int j0, double (&acc)[TT / 16][TT / 16][2],
+                                          NewtonSmem<TT>& sm) {
+  constexpr int FM = TT / 16, HALF = TT / 2;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int wm = warp >> 1, wn = warp & 1;
   auto load = [&](int stage, int k0) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int c = tid + r * kNewtonThreads;          // 512 16-byte chunks per operand
-      const int ar = c >> 3, ac = (c & 7) * 2;         // A: 64 rows x 8 chunks
+    for (int r = 0; r < TT / 16; ++r) {
+      const int c = tid + r * kNewtonThreads;          // TT * 8 16-byte chunks per operand
+      const int ar = c >> 3, ac = (c & 7) * 2;         // A: TT rows x 8 chunks
       cp_async16(&sm.As[stage][ar][ac], A + (size_t)(i0 + ar) * S + k0 + ac);
-      const int br = c >> 5, bc = (c & 31) * 2;        // B: 16 rows x 32 chunks
+      const int br = c / HALF, bc = (c % HALF) * 2;    // B: 16 rows x TT/2 chunks
       cp_async16(&sm.Bs[stage][br][bc], B + (size_t)(k0 + br) * S + j0 + bc);
     }
     cp_async_commit();
   };
   const int nk = S / kBK;
-  // on a diagonal tile the lower-left 32 x 32 block mirrors the upper-right one
+  // on a diagonal tile the lower-left sub-tile mirrors the upper-right one
   const bool idle = (i0 == j0) && wm == 1 && wn == 0;
   load(0, 0);
   for (int kt = 0; kt < nk; ++kt) {
@@ -115,23 +119,23 @@ __device__ __forceinline__ void dmma_tile(const double* __restrict__ A, const do
     const int st = kt & 1;
 #pragma unroll
     for (int kk = 0; kk < kBK && !idle; kk += 4) {
-      double a[4], b[4];
+      double a[FM], b[FM];
 #pragma unroll
-      for (int mi = 0; mi < 4; ++mi) a[mi] = sm.As[st][wm * 32 + mi * 8 + g][kk + t];
+      for (int mi = 0; mi < FM; ++mi) a[mi] = sm.As[st][wm * HALF + mi * 8 + g][kk + t];
 #pragma unroll
-      for (int ni = 0; ni < 4; ++ni) b[ni] = sm.Bs[st][kk + t][wn * 32 + ni * 8 + g];
+      for (int ni = 0; ni < FM; ++ni) b[ni] = sm.Bs[st][kk + t][wn * HALF + ni * 8 + g];
 #pragma unroll
-      for (int mi = 0; mi < 4; ++mi)
+      for (int mi = 0; mi < FM; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) dmma884(acc[mi][ni][0], acc[mi][ni][1], a[mi], b[ni]);
+        for (int ni = 0; ni < FM; ++ni) dmma884(acc[mi][ni][0], acc[mi][ni][1], a[mi], b[ni]);
     }
     __syncthreads();
   }
 }
 
-// How a warp's 32 x 32 block of a tile is stored: on a diagonal tile the
-// lower-left warp computes nothing (its block mirrors the upper-right one);
-// every block off the matrix diagonal is also written transposed.
+// How a warp's sub-tile of a tile is stored: on a diagonal tile the
+// lower-left warp computes nothing (its sub-tile mirrors the upper-right
+// one); every sub-tile off the matrix diagonal is also written transposed.
 __device__ __forceinline__ int warp_weight(int i0, int j0) {
   const int warp = threadIdx.x >> 5, wm = warp >> 1, wn = warp & 1;
   if (i0 != j0) return 2;            // off-diagonal tile: block and mirror
@@ -140,19 +144,21 @@ __device__ __forceinline__ int warp_weight(int i0, int j0) {
 }
 
 // Store the tile to C at (i0, j0) and its mirror image where it has one.
+template <int TT>
 __device__ __forceinline__ void store_sym(double* __restrict__ C, int S, int i0, int j0,
-                                          const double acc[4][4][2]) {
+                                          const double (&acc)[TT / 16][TT / 16][2]) {
+  constexpr int FM = TT / 16, HALF = TT / 2;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int wm = warp >> 1, wn = warp & 1;
   const int wgt = warp_weight(i0, j0);
   if (wgt == 0) return;
 #pragma unroll
-  for (int mi = 0; mi < 4; ++mi)
+  for (int mi = 0; mi < FM; ++mi)
 #pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      const int r = i0 + wm * 32 + mi * 8 + g;
-      const int c = j0 + wn * 32 + ni * 8 + 2 * t;
+    for (int ni = 0; ni < FM; ++ni) {
+      const int r = i0 + wm * HALF + mi * 8 + g;
+      const int c = j0 + wn * HALF + ni * 8 + 2 * t;
       *reinterpret_cast<double2*>(C + (size_t)r * S + c) = make_double2(acc[mi][ni][0], acc[mi][ni][1]);
       if (wgt == 2) {
         C[(size_t)c * S + r] = acc[mi][ni][0];
@@ -505,100 +511,106 @@ __global__ void __launch_bounds__(256) newton_t0_kernel(const NewtonMat* __restr
 //   M_next = T^p M, residual, T <- ((p+1) I - M_next)/p  (launch C)
 // grid: x = upper-triangular tile, y = matrix, z = job.
 // ---------------------------------------------------------------------------
+template <int TT>
 __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
     const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
-  __shared__ NewtonSmem sm;
+  constexpr int FM = TT / 16;
+  __shared__ NewtonSmem<TT> sm;
   const int m = blockIdx.y;
   const int st = w.state[m];
   if (st != kRunning && !(st == kFinal && blockIdx.z == 0)) return;
-  const int T = S / kTile;
+  const int T = S / TT;
   int ti, tj;
   tri_tile(blockIdx.x, T, ti, tj);
   const size_t base = (size_t)m * S * S;
   const double* Tm = w.T + base;
   const double* A = blockIdx.z == 0 ? w.X[it & 1] + base : Tm;
   double* C = blockIdx.z == 0 ? w.X[(it + 1) & 1] + base : w.T2 + base;
-  double acc[4][4][2] = {};
-  dmma_tile(A, Tm, S, ti * kTile, tj * kTile, acc, sm);
+  double acc[FM][FM][2] = {};
+  dmma_tile<TT>(A, Tm, S, ti * TT, tj * TT, acc, sm);
   if (blockIdx.z == 0) {   // X_next = s_k^{1/p} X T
     const double sk = sched_at(w, m, it);
     if (sk != 1.0) {
       const double mu = pow(sk, 1.0 / mats[m].p);
 #pragma unroll
-      for (int mi = 0; mi < 4; ++mi)
+      for (int mi = 0; mi < FM; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) {
+        for (int ni = 0; ni < FM; ++ni) {
           acc[mi][ni][0] *= mu;
           acc[mi][ni][1] *= mu;
         }
     }
   }
-  store_sym(C, S, ti * kTile, tj * kTile, acc);
+  store_sym<TT>(C, S, ti * TT, tj * TT, acc);
 }
 
+template <int TT>
 __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_b_kernel(
     const NewtonMat* __restrict__ mats, int S, NewtonWork w) {
-  __shared__ NewtonSmem sm;
+  constexpr int FM = TT / 16;
+  __shared__ NewtonSmem<TT> sm;
   const int m = blockIdx.y;
   if (w.state[m] != kRunning || mats[m].p != 4) return;
-  const int T = S / kTile;
+  const int T = S / TT;
   int ti, tj;
   tri_tile(blockIdx.x, T, ti, tj);
   const size_t base = (size_t)m * S * S;
-  double acc[4][4][2] = {};
-  dmma_tile(w.T2 + base, w.T2 + base, S, ti * kTile, tj * kTile, acc, sm);
-  store_sym(w.T4 + base, S, ti * kTile, tj * kTile, acc);
+  double acc[FM][FM][2] = {};
+  dmma_tile<TT>(w.T2 + base, w.T2 + base, S, ti * TT, tj * TT, acc, sm);
+  store_sym<TT>(w.T4 + base, S, ti * TT, tj * TT, acc);
 }
 
+template <int TT>
 __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
     const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
-  __shared__ NewtonSmem sm;
+  constexpr int FM = TT / 16, HALF = TT / 2;
+  __shared__ NewtonSmem<TT> sm;
   __shared__ double red[kNewtonThreads / 32];
   const int m = blockIdx.y;
   if (w.state[m] != kRunning) return;
   const int p = mats[m].p;
-  const int T = S / kTile;
+  const int T = S / TT;
   int ti, tj;
   tri_tile(blockIdx.x, T, ti, tj);
   const size_t base = (size_t)m * S * S;
   const double* Tp = (p == 4 ? w.T4 : w.T2) + base;
-  double acc[4][4][2] = {};
-  const int i0 = ti * kTile, j0 = tj * kTile;
-  dmma_tile(Tp, w.M[it & 1] + base, S, i0, j0, acc, sm);
+  double acc[FM][FM][2] = {};
+  const int i0 = ti * TT, j0 = tj * TT;
+  dmma_tile<TT>(Tp, w.M[it & 1] + base, S, i0, j0, acc, sm);
   // M_next = s_k T^p M
   const double sk = sched_at(w, m, it), sn = sched_at(w, m, it + 1);
 #pragma unroll
-  for (int mi = 0; mi < 4; ++mi)
+  for (int mi = 0; mi < FM; ++mi)
 #pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
+    for (int ni = 0; ni < FM; ++ni) {
       acc[mi][ni][0] *= sk;
       acc[mi][ni][1] *= sk;
     }
-  store_sym(w.M[(it + 1) & 1] + base, S, i0, j0, acc);
+  store_sym<TT>(w.M[(it + 1) & 1] + base, S, i0, j0, acc);
   // residual (valid corner) and the next T = ((p+1) I - s_{k+1} M_next) / p
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int wm = warp >> 1, wn = warp & 1;
   const int n = mats[m].size;
   const double pinv = 1.0 / p;
-  const double wgt = warp_weight(i0, j0);   // 0: idle block, 2: block and mirror
+  const double wgt = warp_weight(i0, j0);   // 0: idle sub-tile, 2: sub-tile and mirror
   double dev = 0.0, f2 = 0.0;
 #pragma unroll
-  for (int mi = 0; mi < 4; ++mi)
+  for (int mi = 0; mi < FM; ++mi)
 #pragma unroll
-    for (int ni = 0; ni < 4; ++ni)
+    for (int ni = 0; ni < FM; ++ni)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int r = i0 + wm * 32 + mi * 8 + g;
-        const int c = j0 + wn * 32 + ni * 8 + 2 * t + e;
+        const int r = i0 + wm * HALF + mi * 8 + g;
+        const int c = j0 + wn * HALF + ni * 8 + 2 * t + e;
         const double d = (r == c) ? 1.0 : 0.0;
         double x = (wgt > 0 && r < n && c < n) ? fabs(acc[mi][ni][e] - d) : 0.0;
         if (!(x <= DBL_MAX)) x = INFINITY;
         dev = fmax(dev, x);
-        f2 += wgt * x * x;                       // mirrored blocks count twice
+        f2 += wgt * x * x;                       // mirrored sub-tiles count twice
         acc[mi][ni][e] = ((p + 1) * d - sn * acc[mi][ni][e]) * pinv;
       }
-  store_sym(w.T + base, S, i0, j0, acc);
+  store_sym<TT>(w.T + base, S, i0, j0, acc);
   dev = block_max(dev, red);
   f2 = block_sum(f2, red);
   if (threadIdx.x == 0) {
@@ -643,9 +655,13 @@ __global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, Ne
     w.state[m] = st;
     alive += (st == kRunning || st == kFinal);
   }
-  // number of threads still holding a running matrix: zero iff none runs
-  alive = __syncthreads_count(alive);
-  if (threadIdx.x == 0) w.count[k & 1] = alive;
+  // number of matrices still running (or with their X-only step left)
+  __shared__ int total;
+  if (threadIdx.x == 0) total = 0;
+  __syncthreads();
+  if (alive) atomicAdd(&total, alive);
+  __syncthreads();
+  if (threadIdx.x == 0) w.count[k & 1] = total;
 }
 
 __global__ void newton_reset_kernel(int nm, NewtonWork w) {
@@ -718,21 +734,30 @@ void launch_newton_t0(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaSt
   newton_t0_kernel<<<dim3(S, nm), 256, 0, s>>>(mats, S, w);
 }
 
-static int num_tri(int S) {
-  const int T = S / kTile;
+static int num_tri(int S, int tile) {
+  const int T = S / tile;
   return T * (T + 1) / 2;
 }
 
-void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s) {
-  newton_step_a_kernel<<<dim3(num_tri(S), nm, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
+  if (tile == 32)
+    newton_step_a_kernel<32><<<dim3(num_tri(S, 32), nm, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+  else
+    newton_step_a_kernel<64><<<dim3(num_tri(S, 64), nm, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
 }
 
-void launch_newton_step_b(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {
-  newton_step_b_kernel<<<dim3(num_tri(S), nm), kNewtonThreads, 0, s>>>(mats, S, w);
+void launch_newton_step_b(const NewtonMat* mats, int nm, int S, int tile, NewtonWork w, cudaStream_t s) {
+  if (tile == 32)
+    newton_step_b_kernel<32><<<dim3(num_tri(S, 32), nm), kNewtonThreads, 0, s>>>(mats, S, w);
+  else
+    newton_step_b_kernel<64><<<dim3(num_tri(S, 64), nm), kNewtonThreads, 0, s>>>(mats, S, w);
 }
 
-void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, NewtonWork w, cudaStream_t s) {
-  newton_step_c_kernel<<<dim3(num_tri(S), nm), kNewtonThreads, 0, s>>>(mats, S, it, w);
+void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
+  if (tile == 32)
+    newton_step_c_kernel<32><<<dim3(num_tri(S, 32), nm), kNewtonThreads, 0, s>>>(mats, S, it, w);
+  else
+    newton_step_c_kernel<64><<<dim3(num_tri(S, 64), nm), kNewtonThreads, 0, s>>>(mats, S, it, w);
 }
 
 void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s) {

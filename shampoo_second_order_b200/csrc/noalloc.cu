@@ -196,9 +196,9 @@ extern "C" shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, f
       int alive = 0;
       e = read_int(&w.count[0], &alive, st);
       for (int it = 0; it < max_iters && alive && e == cudaSuccess; ++it) {
-        launch_newton_step_a(mats, nm, S, it, w, st);
-        if (p == 4) launch_newton_step_b(mats, nm, S, w, st);
-        launch_newton_step_c(mats, nm, S, it, w, st);
+        launch_newton_step_a(mats, nm, S, it, 64, w, st);
+        if (p == 4) launch_newton_step_b(mats, nm, S, 64, w, st);
+        launch_newton_step_c(mats, nm, S, it, 64, w, st);
         launch_newton_check(nm, it + 1, tol, max_iters, w, st);
         e = read_int(&w.count[(it + 1) & 1], &alive, st);
       }
