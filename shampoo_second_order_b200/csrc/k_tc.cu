@@ -199,7 +199,10 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
           break;
         }
         uint8_t* st = smem + s * stage_bytes;
-        tc::mbar_expect_tx(&full[s], stage_bytes);
+        // a diagonal statistics tile multiplies a panel by itself: its B
+        // operand is the A panel already in the stage
+        const bool diag = (MODE == kStats) && i0 == j0;
+        tc::mbar_expect_tx(&full[s], diag ? nA * kBoxBytes : stage_bytes);
         const int k0 = kt * kBKe;
         for (int pa = 0; pa < nA; ++pa) {
           uint8_t* dst = st + pa * kBoxBytes;
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nblk + blk);
           }
         }
-        for (int pb = 0; pb < nB; ++pb) {
+        for (int pb = 0; pb < nB && !diag; ++pb) {
           uint8_t* dst = st + (nA + pb) * kBoxBytes;
           if (MODE == kStats && isR) {
             tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
@@ -236,6 +239,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       if (x.skip) continue;
       const int a_mn = (MODE == kStats) ? x.isR : 0;
       const int b_mn = (MODE == kStats) ? x.isR : (MODE == kApplyP);
+      const bool diag = (MODE == kStats) && x.i0 == x.j0;   // B operand = the A panel
       const uint32_t idesc = tc::idesc_bf16(kTM, kTM, a_mn, b_mn);
       const int acc = i & 1;
       if (i >= 2 && !tc::mbar_wait(&tempty[acc], ((i >> 1) - 1) & 1)) {
@@ -263,7 +267,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             const int pa = (pas >> (2 * q)) & 3;
             const int pb = (pbs >> (2 * q)) & 3;
             const uint32_t sa = st + pa * kBoxBytes;
-            const uint32_t sb = st + (nA + pb) * kBoxBytes;
+            const uint32_t sb = st + (diag ? pb : nA + pb) * kBoxBytes;
             const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
                                      : tc::smem_desc(sa + kk * 32, 16, 1024);
             const uint64_t db = b_mn ? tc::smem_desc(sb + kk * 2048, 8192, 1024)

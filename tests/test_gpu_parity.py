@@ -547,3 +547,34 @@ def test_async_roots_busy_and_sync_refused():
     assert rel(X_async, X_sync1) <= 1e-6
     assert busy
     opt.close()
+
+
+# --------------------------------------------------------------------------
+# block-sharded data parallelism through the CUDA library (one process: the
+# owner plan gives every parameter to rank 0; the packing of gradients and
+# weights around the library context is what runs)
+# --------------------------------------------------------------------------
+def test_sharded_single_rank_matches_oracle():
+    from shampoo_second_order_b200.sharded import ShardedShampoo
+    shapes = [(200, 130), (64, 64), (19, 200), (130,), (1, 77)]
+    b, beta2, eps, lr, gstd = 64, 0.99, 1e-6, 0.1, 1e-2
+    opt = ShardedShampoo(shapes, b, beta2, eps, 4, 1, 0.5, "f32", root_interval=3)
+    o = ShampooOracle(shapes, b, beta2, eps, 4, 1, 0.5)
+    W0 = wl.make_params(shapes, 12)
+    Wd = [torch.from_numpy(w).cuda() for w in W0]
+    Wo = [w.astype(np.float64) for w in W0]
+    worst = 0.0
+    for t in range(6):
+        g = wl.make_grads(shapes, 12, t, gstd, "f32")
+        prev_d = [w.cpu().numpy().astype(np.float64) for w in Wd]
+        prev_o = Wo
+        opt.step(Wd, [to_dev(x, "f32") for x in g], lr, t % 3 == 0)
+        Wo = o.step(Wo, g, lr, t % 3 == 0)
+        torch.cuda.synchronize()
+        for i, s in enumerate(shapes):
+            wd = Wd[i].cpu().numpy().astype(np.float64)
+            for sl in pieces(s, b):
+                worst = max(worst, rel((wd - prev_d[i])[sl], (Wo[i] - prev_o[i])[sl]))
+    assert opt.mine == list(range(len(shapes)))
+    assert worst <= STEP_TOL, worst
+    opt.close()
