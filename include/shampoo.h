@@ -398,6 +398,18 @@ shampoo_status shampoo_plan_shards(int nparams, const int64_t* shapes,
                                    int root_interval, int nranks, int32_t* owner,
                                    double* rank_cost);
 
+/*
+ * shampoo_selftest_stalled_wait -- failure-path check: launches one warp
+ * that waits, through the same bounded mbarrier wait every tensor-core
+ * pipeline of the library uses, on a barrier phase that nothing completes.
+ * The wait gives up after about 2^31 clock cycles (about a second), records
+ * the timeout the way a stalled pipeline does and the kernel returns, so the
+ * call ends with SHAMPOO_ECUDA ("timed out waiting on its pipeline") and the
+ * CUDA context stays usable.  A test of the error path: no fault, no hang.
+ * stream: caller-owned cudaStream_t.  Allocates and frees 4 bytes.
+ */
+shampoo_status shampoo_selftest_stalled_wait(void* stream);
+
 /* Library version, "MAJOR.MINOR.PATCH". */
 const char* shampoo_version(void);
 

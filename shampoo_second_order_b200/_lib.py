@@ -52,6 +52,7 @@ SIGNATURES = {
                                                        C.c_double, C.c_int, _P, _P]),
     "shampoo_plan_shards": (C.c_int, [C.c_int, C.POINTER(C.c_int64), C.POINTER(C.c_int32), C.c_int, C.c_int,
                                       C.c_int, C.POINTER(C.c_int32), C.POINTER(C.c_double)]),
+    "shampoo_selftest_stalled_wait": (C.c_int, [_P]),
     "shampoo_version": (C.c_char_p, []),
 }
 

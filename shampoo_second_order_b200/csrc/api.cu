@@ -1053,6 +1053,21 @@ shampoo_status shampoo_set_one_sided(shampoo_ctx* ctx, int param, int side) {
   return SHAMPOO_OK;
 }
 
+shampoo_status shampoo_selftest_stalled_wait(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* d = nullptr;
+  int h = 0;
+  cudaError_t e = cudaMalloc(&d, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemsetAsync(d, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = launch_stalled_wait(d, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, d, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (d) cudaFree(d);
+  if (e != cudaSuccess) return fail(nullptr, SHAMPOO_ECUDA, std::string("stalled-wait self-test: ") + cudaGetErrorString(e));
+  if (h) return fail(nullptr, SHAMPOO_ECUDA, "a tensor-core kernel timed out waiting on its pipeline");
+  return SHAMPOO_OK;
+}
+
 int shampoo_num_matrices(const shampoo_ctx* ctx) { return ctx ? ctx->nmat : 0; }
 
 shampoo_status shampoo_matrix_info(const shampoo_ctx* ctx, int index, int* size, int* root_p) {

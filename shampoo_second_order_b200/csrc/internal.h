@@ -62,6 +62,8 @@ struct TcMaps {
 cudaError_t launch_gather(const BlockDesc* blocks, int nblk, const void* const* gptr, int bf16,
                           int* flags, int S, uint16_t* out, cudaStream_t s);
 cudaError_t launch_split(const float* x, int64_t n, uint16_t* out, cudaStream_t s);
+// a wait that runs out: sets *err to the timeout code after about a second
+cudaError_t launch_stalled_wait(int* err, cudaStream_t s);
 cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
                             int nmat, int S, int planes_g, float beta2, float* stats, int* err,
                             cudaStream_t s);

@@ -603,6 +603,23 @@ cudaError_t launch_gather(const BlockDesc* blocks, int nblk, const void* const* 
   return cudaGetLastError();
 }
 
+// One warp waits, through the pipelines' bounded wait, on a barrier phase
+// that nothing completes; the give-up lands in *err like a stalled pipeline's.
+__global__ void stalled_wait_kernel(int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0 && !tc::mbar_wait(&bar, 0)) atomicExch(err, tc::kErrTimeout);
+}
+
+cudaError_t launch_stalled_wait(int* err, cudaStream_t s) {
+  stalled_wait_kernel<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_split(const float* x, int64_t n, uint16_t* out, cudaStream_t s) {
   split_kernel<<<1184, 256, 0, s>>>(x, n, out);
   return cudaGetLastError();

@@ -578,3 +578,19 @@ def test_sharded_single_rank_matches_oracle():
     assert opt.mine == list(range(len(shapes)))
     assert worst <= STEP_TOL, worst
     opt.close()
+
+
+def test_stalled_pipeline_wait_is_reported_and_the_context_survives():
+    """A bounded wait that nothing satisfies ends in about a second with the
+    pipeline-timeout status (no hang), and the device keeps working."""
+    import time
+    from shampoo_second_order_b200 import _lib, batched_inverse_root
+    t0 = time.time()
+    st = _lib.lib().shampoo_selftest_stalled_wait(None)
+    assert st == _lib.ECUDA
+    assert "timed out" in _lib.lib().shampoo_last_error(None).decode()
+    assert time.time() - t0 < 30
+    A = torch.eye(64, device="cuda").mul_(4.0).unsqueeze(0).contiguous()
+    X, iters = batched_inverse_root(A, 2, 1e-6)
+    assert int(iters[0]) >= 0
+    assert torch.allclose(X[0], torch.eye(64, device="cuda") * (4.0 + 1e-6) ** -0.5)
