@@ -150,3 +150,53 @@ def test_sharded_step_matches_one_oracle_on_mean_gradients():
         assert nbytes > 0
         owned += mine
     assert sorted(owned) == list(range(len(SHAPES)))   # every parameter has exactly one owner
+
+
+def _dying_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    from shampoo_second_order_b200.sharded import ShardedShampoo
+    c = CFG
+    opt = ShardedShampoo(SHAPES, c["b"], c["beta2"], c["eps"], graft=c["graft"], momentum=c["mu"],
+                         root_interval=c["interval"],
+                         make_local=lambda sh: OracleLocal(sh, c["b"], c["beta2"], c["eps"], c["graft"], c["mu"]))
+    W = [torch.from_numpy(w.astype(np.float32)) for w in wl.make_params(SHAPES, 5)]
+    g = [torch.from_numpy(x) for x in _rank_grads(rank, 0)]
+    opt.step(W, g, c["lr"], True)                 # one good step together
+    if rank == 1:
+        q.put((rank, "died"))
+        q.close()
+        q.join_thread()                            # the message is out before the process goes
+        os._exit(3)                                # leaves between steps, nothing in flight
+    import time
+    t0 = time.time()
+    try:
+        opt.step(W, g, c["lr"], False)
+        q.put((rank, "no error"))
+    except Exception as e:                         # the collective reports the missing rank
+        q.put((rank, "error after %.1f s: %s" % (time.time() - t0, type(e).__name__)))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_sharded_step_reports_a_dead_rank():
+    """A rank that leaves between steps: the survivor's next reduce-scatter
+    ends with an error from the process group (within its 10 s timeout), not
+    a hang."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert out[1] == "died"
+    assert out[0].startswith("error after"), out[0]
+    assert float(out[0].split()[2]) < 60
