@@ -23,6 +23,7 @@
 //
 // Kernels:
 //   ozaki_split  per row: exponent and qs int8 slice planes of a float64 iterate
+//                (T's slices come from M, T = ((p+1) I - s M) / p, in the same pass)
 //   ozaki_gemm   persistent, warp-specialised: lane 0 of warp 0 loads the
 //                slice planes by TMA (a stage = one slice of A's 128-row
 //                tile and of B's 64-row tile over 64 K), lane 0 of warp 1
@@ -60,58 +61,46 @@ constexpr uint32_t kIdesc = tc::idesc_s8(kTileM, kTileN);
 struct SplitJobs {
   const double* src[2];   // float64 [qcap][S][S]
   int set[2];
+  int with_t[2];          // 1: src is M; also slice T = ((p+1) I - s_it M) / p into set kOzT
+  int it;                 // schedule index of that T
 };
 
-// grid: x = group of 8 rows, y = matrix, z = job.  One warp per row; lane l
-// holds the columns 128 i + 4 l .. + 3.
-__global__ void __launch_bounds__(256) ozaki_split_kernel(const NewtonMat* __restrict__ mats, int S,
-                                                          SplitJobs jobs, NewtonWork w) {
-  const int m = blockIdx.y;
-  if (w.state[m] != kRunning) return;
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (r >= S) return;
-  const int set = jobs.set[blockIdx.z];
-  const double* row = jobs.src[blockIdx.z] + (size_t)m * S * S + (size_t)r * S;
-  const int qs = w.qs;
-  double v[32];
+// Exponent and slices of one row held as 4 NCH values per lane (columns
+// 128 i + 4 lane .. + 3); `val` maps a stored value to the one to slice.
+template <int NCH, class F>
+__device__ __forceinline__ void slice_row(const double (&v)[4 * NCH], int S, int c0, int lane, int qs,
+                                          int8_t* q0, size_t plane, int* exp_out, F val) {
   double mx = 0.0;
   bool bad = false;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = 128 * i + 4 * lane;
-    if (c < S) {
-      const double2 a = *reinterpret_cast<const double2*>(row + c);
-      const double2 b = *reinterpret_cast<const double2*>(row + c + 2);
-      v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = b.x; v[4 * i + 3] = b.y;
+  for (int i = 0; i < NCH; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        bad |= !(fabs(v[4 * i + j]) <= DBL_MAX);
-        mx = fmax(mx, fabs(v[4 * i + j]));
+    for (int j = 0; j < 4; ++j) {
+      const int c = 128 * i + 4 * lane + j;
+      if (c < S) {
+        const double x = val(v[4 * i + j], c);
+        bad |= !(fabs(x) <= DBL_MAX);
+        mx = fmax(mx, fabs(x));
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[4 * i + j] = 0.0;
     }
-  }
   mx = warp_max(mx);
   bad = __any_sync(0xffffffffu, bad);
   int e = 0;
-  if (!bad && mx > 0.0) frexp(mx, &e);        // mx = f 2^e, f in [0.5, 1): every |v| < 2^e
+  if (!bad && mx > 0.0) frexp(mx, &e);        // mx = f 2^e, f in [0.5, 1): every |x| < 2^e
   // a row far below the float64 range of its neighbours counts as zero
   const bool zero = bad || mx == 0.0 || e < -900;
   const double scale = zero ? 0.0 : ldexp(1.0, 7 * qs - e);
-  int8_t* q0 = w.q + ((size_t)set * qs * w.qcap + m) * S * S + (size_t)r * S;
-  const size_t plane = (size_t)w.qcap * S * S;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < NCH; ++i) {
     const int c = 128 * i + 4 * lane;
     if (c >= S) continue;
     unsigned long long f[4];
     bool neg[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      f[j] = (unsigned long long)(fabs(v[4 * i + j]) * scale);   // < 2^{7 qs}: exact scaling, truncated
-      neg[j] = v[4 * i + j] < 0.0;
+      const double x = val(v[4 * i + j], c + j);
+      f[j] = (unsigned long long)(fabs(x) * scale);   // < 2^{7 qs}: exact scaling, truncated
+      neg[j] = x < 0.0;
     }
     for (int k = 0; k < qs; ++k) {
       const int sh = 7 * (qs - 1 - k);
@@ -125,7 +114,44 @@ __global__ void __launch_bounds__(256) ozaki_split_kernel(const NewtonMat* __res
       *reinterpret_cast<uint32_t*>(q0 + k * plane + c) = word;
     }
   }
-  if (lane == 0) w.qe[((size_t)set * w.qcap + m) * S + r] = bad ? kBadExp : (zero ? 0 : e);
+  if (lane == 0) *exp_out = bad ? kBadExp : (zero ? 0 : e);
+}
+
+// grid: x = group of 8 rows, y = matrix, z = job.  One warp per row, S <= 128 NCH.
+template <int NCH>
+__global__ void __launch_bounds__(256) ozaki_split_kernel(const NewtonMat* __restrict__ mats, int S,
+                                                          SplitJobs jobs, NewtonWork w) {
+  const int m = blockIdx.y;
+  if (w.state[m] != kRunning) return;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= S) return;
+  const int z = blockIdx.z, set = jobs.set[z];
+  const double* row = jobs.src[z] + (size_t)m * S * S + (size_t)r * S;
+  const int qs = w.qs;
+  double v[4 * NCH];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const int c = 128 * i + 4 * lane;
+    if (c < S) {
+      const double2 a = *reinterpret_cast<const double2*>(row + c);
+      const double2 b = *reinterpret_cast<const double2*>(row + c + 2);
+      v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = b.x; v[4 * i + 3] = b.y;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * i + j] = 0.0;
+    }
+  }
+  const size_t plane = (size_t)w.qcap * S * S;
+  int8_t* q0 = w.q + ((size_t)set * qs * w.qcap + m) * S * S + (size_t)r * S;
+  slice_row<NCH>(v, S, 0, lane, qs, q0, plane, &w.qe[((size_t)set * w.qcap + m) * S + r],
+                 [](double x, int) { return x; });
+  if (jobs.with_t[z]) {   // T from M: its digits in set kOzT, without a float64 copy of T
+    const int p = mats[m].p;
+    const double sn = newton_sched(w, m, jobs.it), pinv = 1.0 / p;
+    int8_t* qt = w.q + ((size_t)kOzT * qs * w.qcap + m) * S * S + (size_t)r * S;
+    slice_row<NCH>(v, S, 0, lane, qs, qt, plane, &w.qe[((size_t)kOzT * w.qcap + m) * S + r],
+                   [&](double x, int c) { return ((p + 1) * (r == c ? 1.0 : 0.0) - sn * x) * pinv; });
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -414,9 +440,6 @@ __global__ void __launch_bounds__(192, 1) ozaki_gemm_kernel(const __grid_constan
             dev = fmax(dev, xd);
             f2 += (r == col ? 1.0 : 2.0) * xd * xd;   // an entry above the diagonal counts for its mirror too
           }
-          const double tn = ((p + 1) * dl - sn * v) * pinv;   // next T = ((p+1) I - s_{k+1} M_next) / p
-          w.T[base + (size_t)r * S + col] = tn;
-          if (r < col) w.T[base + (size_t)col * S + r] = tn;
         }
       };
 #pragma unroll
@@ -476,23 +499,39 @@ cudaError_t launch_gemm(const OzakiMaps& maps, const OzArgs& a, int ntiles, int 
 
 }  // namespace
 
+template <int NCH>
+void launch_split_jobs(const NewtonMat* mats, int nm, int S, const SplitJobs& jobs, int nj, NewtonWork w,
+                       cudaStream_t s) {
+  ozaki_split_kernel<NCH><<<dim3((S + 7) / 8, nm, nj), 256, 0, s>>>(mats, S, jobs, w);
+}
+
 cudaError_t launch_ozaki_split(const NewtonMat* mats, int nm, int S, int it, unsigned sets, NewtonWork w,
                                cudaStream_t s) {
-  // the float64 source of each set at step `it` (X and M: the buffers step it wrote)
+  // the float64 source of each set at step `it` (X and M: the buffers step it
+  // wrote); T, when asked together with M, comes from M in the same pass
   const double* src[kOzSets] = {w.X[it & 1], w.T, w.T2, w.T4, w.M[it & 1]};
+  const bool t_from_m = (sets >> kOzM & 1u) && (sets >> kOzT & 1u);
+  if (t_from_m) sets &= ~(1u << kOzT);
   SplitJobs jobs{};
+  jobs.it = it;
   int nj = 0;
+  auto flush = [&] {
+    if (!nj) return;
+    if (S <= 128) launch_split_jobs<1>(mats, nm, S, jobs, nj, w, s);
+    else if (S <= 256) launch_split_jobs<2>(mats, nm, S, jobs, nj, w, s);
+    else if (S <= 512) launch_split_jobs<4>(mats, nm, S, jobs, nj, w, s);
+    else launch_split_jobs<8>(mats, nm, S, jobs, nj, w, s);
+    nj = 0;
+  };
   for (int z = 0; z < kOzSets; ++z) {
     if (!(sets >> z & 1u)) continue;
-    if (nj == 2) {
-      ozaki_split_kernel<<<dim3((S + 7) / 8, nm, nj), 256, 0, s>>>(mats, S, jobs, w);
-      nj = 0;
-    }
+    if (nj == 2) flush();
     jobs.src[nj] = src[z];
     jobs.set[nj] = z;
+    jobs.with_t[nj] = (z == kOzM && t_from_m) ? 1 : 0;
     ++nj;
   }
-  if (nj) ozaki_split_kernel<<<dim3((S + 7) / 8, nm, nj), 256, 0, s>>>(mats, S, jobs, w);
+  flush();
   return cudaGetLastError();
 }
 
