@@ -119,7 +119,7 @@ __device__ __forceinline__ void slice_row(const double (&v)[4 * NCH], int S, int
 
 // grid: x = group of 8 rows, y = matrix, z = job.  One warp per row, S <= 128 NCH.
 template <int NCH>
-__global__ void __launch_bounds__(256) ozaki_split_kernel(const NewtonMat* __restrict__ mats, int S,
+__global__ void __launch_bounds__(256, NCH <= 4 ? 3 : 1) ozaki_split_kernel(const NewtonMat* __restrict__ mats, int S,
                                                           SplitJobs jobs, NewtonWork w) {
   const int m = blockIdx.y;
   if (w.state[m] != kRunning) return;
