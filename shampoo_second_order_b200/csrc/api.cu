@@ -123,6 +123,10 @@ void run(Profiler* pr, const char* name, cudaStream_t s, F&& f) {
 
 struct shampoo_ctx {
   cudaStream_t stream = nullptr;
+  // the small 1-D kernels run beside the tensor-core GEMMs on this stream
+  // (same priority as `stream`), forked and joined with events
+  cudaStream_t aux = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   int nparams = 0, b = 0, S = 0, p = 4, graft = 1, bf16 = 0;
   float beta2 = 1.f, eps = 1e-6f, mu = 0.f;
   double tol = 1e-6;
@@ -629,6 +633,12 @@ void shampoo_destroy(shampoo_ctx* ctx) {
     cudaStreamDestroy(ctx->side);
   }
   if (ctx->ev_submit) cudaEventDestroy(ctx->ev_submit);
+  if (ctx->aux) {
+    cudaStreamSynchronize(ctx->aux);
+    cudaStreamDestroy(ctx->aux);
+  }
+  if (ctx->ev_fork) cudaEventDestroy(ctx->ev_fork);
+  if (ctx->ev_join) cudaEventDestroy(ctx->ev_join);
   cudaStreamSynchronize(ctx->stream);
   for (void* q : ctx->allocs) cudaFree(q);
   if (ctx->h_count) cudaFreeHost(ctx->h_count);
@@ -765,6 +775,11 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
     return fail(nullptr, SHAMPOO_ENOMEM, std::string("device allocation failed: ") + cudaGetErrorString(e));
   }
   e = cudaMallocHost(&ctx->h_count, 2 * sizeof(int));
+  int prio = 0;
+  if (e == cudaSuccess) e = cudaStreamGetPriority(ctx->stream, &prio);
+  if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ctx->aux, cudaStreamNonBlocking, prio);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->stats, 0, ctx->nmat * slot * sizeof(float), ctx->stream);
@@ -816,6 +831,15 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
     shampoo_status gs = gather(ctx, grads, true);
     if (gs != SHAMPOO_OK) return gs;
   }
+  if (nseg) {   // the 1-D statistics beside the block work (disjoint slots)
+    CK(cudaEventRecord(ctx->ev_fork, s));
+    CK(cudaStreamWaitEvent(ctx->aux, ctx->ev_fork, 0));
+    run(pr, "stats_segments", ctx->aux, [&] {
+      launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
+                            ctx->beta2, ctx->stats, ctx->S, ctx->aux);
+    });
+    CK(cudaEventRecord(ctx->ev_join, ctx->aux));
+  }
   if (ctx->graft) {
     CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), s));
     run(pr, "diag_update", s, [&] {
@@ -832,11 +856,7 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
     });
     if (e != cudaSuccess) return cuda_fail(ctx, e, "stats_tc");
   }
-  if (nseg)
-    run(pr, "stats_segments", s, [&] {
-      launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
-                            ctx->beta2, ctx->stats, ctx->S, s);
-    });
+  if (nseg) CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
   CK(cudaGetLastError());
   ctx->stats_done = true;
   return SHAMPOO_OK;
@@ -933,6 +953,16 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
   const int nseg = (int)ctx->segs.size();
   Profiler* pr = &ctx->prof;
   CK(cudaMemsetAsync(ctx->p2, 0, ctx->nparams * sizeof(double), s));
+  if (nseg) {   // the 1-D preconditioning beside the block GEMMs (disjoint parameters)
+    CK(cudaEventRecord(ctx->ev_fork, s));
+    CK(cudaStreamWaitEvent(ctx->aux, ctx->ev_fork, 0));
+    run(pr, "precond_seg", ctx->aux, [&] {
+      launch_precondition_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_params, ctx->d_gptr,
+                                   ctx->bf16, ctx->flags, ctx->roots, ctx->S, ctx->P, ctx->p2,
+                                   ctx->aux);
+    });
+    CK(cudaEventRecord(ctx->ev_join, ctx->aux));
+  }
   bool same = ctx->stats_from.size() == (size_t)ctx->nparams;
   for (int i = 0; same && i < ctx->nparams; ++i) same = ctx->stats_from[i] == grads[i];
   if (ctx->graft && !same) {   // ||D||^2 of these gradients against the current a
@@ -957,11 +987,7 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
     });
     if (e != cudaSuccess) return cuda_fail(ctx, e, "apply_p_tc");
   }
-  if (nseg)
-    run(pr, "precond_seg", s, [&] {
-      launch_precondition_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_params, ctx->d_gptr,
-                                   ctx->bf16, ctx->flags, ctx->roots, ctx->S, ctx->P, ctx->p2, s);
-    });
+  if (nseg) CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
   run(pr, "update", s, [&] {
     launch_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_wptr, ctx->flags, ctx->P, ctx->d2,
                   ctx->p2, ctx->graft, ctx->mu, lr, ctx->mom, s);
