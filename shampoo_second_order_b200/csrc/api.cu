@@ -123,10 +123,11 @@ void run(Profiler* pr, const char* name, cudaStream_t s, F&& f) {
 
 struct shampoo_ctx {
   cudaStream_t stream = nullptr;
-  // the small 1-D kernels run beside the tensor-core GEMMs on this stream
-  // (same priority as `stream`), forked and joined with events
+  // the accumulator and the small 1-D kernels run beside the tensor-core
+  // GEMMs on this stream (same priority as `stream`), forked and joined with
+  // events
   cudaStream_t aux = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_mid = nullptr, ev_join = nullptr;
   int nparams = 0, b = 0, S = 0, p = 4, graft = 1, bf16 = 0;
   float beta2 = 1.f, eps = 1e-6f, mu = 0.f;
   double tol = 1e-6;
@@ -638,6 +639,7 @@ void shampoo_destroy(shampoo_ctx* ctx) {
     cudaStreamDestroy(ctx->aux);
   }
   if (ctx->ev_fork) cudaEventDestroy(ctx->ev_fork);
+  if (ctx->ev_mid) cudaEventDestroy(ctx->ev_mid);
   if (ctx->ev_join) cudaEventDestroy(ctx->ev_join);
   cudaStreamSynchronize(ctx->stream);
   for (void* q : ctx->allocs) cudaFree(q);
@@ -779,6 +781,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   if (e == cudaSuccess) e = cudaStreamGetPriority(ctx->stream, &prio);
   if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ctx->aux, cudaStreamNonBlocking, prio);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_mid, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming);
@@ -816,37 +819,41 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   shampoo_status st = set_pointers(ctx, grads, nullptr);
   if (st != SHAMPOO_OK) return st;
-  cudaStream_t s = ctx->stream;
+  cudaStream_t s = ctx->stream, x = ctx->aux;
   const int nch = (int)ctx->chunks.size();
   const int nblk = (int)ctx->blocks.size(), nseg = (int)ctx->segs.size();
   Profiler* pr = &ctx->prof;
   CK(cudaMemsetAsync(ctx->flags, 0, ctx->nparams * sizeof(int), s));
-  // the non-finite check: 1-D gradients here, 2-D ones inside the gather
+  // Two streams: the gather and the block statistics on `stream`; the 1-D
+  // non-finite check, the Adagrad accumulator and the 1-D statistics on the
+  // auxiliary stream beside them.  The accumulator waits for the gather,
+  // which flags non-finite 2-D gradients.
+  CK(cudaEventRecord(ctx->ev_fork, s));
+  CK(cudaStreamWaitEvent(x, ctx->ev_fork, 0));
   const int nch1 = (int)ctx->chunks1d.size();
   if (nch1)
-    run(pr, "check_finite", s, [&] {
-      launch_check_finite(ctx->d_chunks1d, nch1, ctx->d_gptr, ctx->bf16, ctx->flags, s);
+    run(pr, "check_finite", x, [&] {
+      launch_check_finite(ctx->d_chunks1d, nch1, ctx->d_gptr, ctx->bf16, ctx->flags, x);
     });
   if (nblk) {
     shampoo_status gs = gather(ctx, grads, true);
     if (gs != SHAMPOO_OK) return gs;
   }
-  if (nseg) {   // the 1-D statistics beside the block work (disjoint slots)
-    CK(cudaEventRecord(ctx->ev_fork, s));
-    CK(cudaStreamWaitEvent(ctx->aux, ctx->ev_fork, 0));
-    run(pr, "stats_segments", ctx->aux, [&] {
-      launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
-                            ctx->beta2, ctx->stats, ctx->S, ctx->aux);
-    });
-    CK(cudaEventRecord(ctx->ev_join, ctx->aux));
-  }
+  CK(cudaEventRecord(ctx->ev_mid, s));
+  CK(cudaStreamWaitEvent(x, ctx->ev_mid, 0));
   if (ctx->graft) {
-    CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), s));
-    run(pr, "diag_update", s, [&] {
+    CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), x));
+    run(pr, "diag_update", x, [&] {
       launch_diag_update(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags,
-                         ctx->beta2, ctx->eps, ctx->a, ctx->d2, s);
+                         ctx->beta2, ctx->eps, ctx->a, ctx->d2, x);
     });
   }
+  if (nseg)   // the 1-D statistics: slots disjoint from the blocks'
+    run(pr, "stats_segments", x, [&] {
+      launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
+                            ctx->beta2, ctx->stats, ctx->S, x);
+    });
+  CK(cudaEventRecord(ctx->ev_join, x));
   ctx->stats_from.assign(grads, grads + ctx->nparams);
   if (nblk) {
     cudaError_t e = cudaSuccess;
@@ -856,7 +863,7 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
     });
     if (e != cudaSuccess) return cuda_fail(ctx, e, "stats_tc");
   }
-  if (nseg) CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
+  CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
   CK(cudaGetLastError());
   ctx->stats_done = true;
   return SHAMPOO_OK;
