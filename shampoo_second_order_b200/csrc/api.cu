@@ -309,8 +309,9 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
       for (const auto& m : list) has_p4 |= (m.p == 4);
       run(pr, "newton_reset", st, [&] { launch_newton_reset(nm, w, st); });
       run(pr, "newton_bound", st, [&] {
-        launch_newton_bound(A, a_stride, lda, upper, d, nm, S, eps, attempt, w, st);
+        launch_newton_bound_partial(A, a_stride, lda, upper, d, nm, S, eps, w, st);
       });
+      run(pr, "newton_bound_final", st, [&] { launch_newton_bound_final(d, nm, S, eps, attempt, w, st); });
       run(pr, "newton_init", st, [&] { launch_newton_init(A, a_stride, lda, upper, d, nm, S, w, st); });
       run(pr, "newton_lanczos", st, [&] { launch_newton_lanczos(d, nm, S, w, st); });
       run(pr, "newton_t0", st, [&] { launch_newton_t0(d, nm, S, w, st); });

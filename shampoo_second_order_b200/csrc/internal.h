@@ -131,6 +131,11 @@ void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s);
 // of a lower tile is read from (c, r).
 void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
                          int nm, int S, float eps, int attempt, NewtonWork w, cudaStream_t s);
+// the two kernels of launch_newton_bound: partial sums over row bands, then c^p
+void launch_newton_bound_partial(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                                 int nm, int S, float eps, NewtonWork w, cudaStream_t s);
+void launch_newton_bound_final(const NewtonMat* mats, int nm, int S, float eps, int attempt, NewtonWork w,
+                               cudaStream_t s);
 void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
                         int nm, int S, NewtonWork w, cudaStream_t s);
 // Lanczos estimate of M0's spectrum and the scaling schedule, then T0.

@@ -712,12 +712,22 @@ void launch_newton_reset(int nm, NewtonWork w, cudaStream_t s) {
 
 // c^p goes to the first nm doubles of T2, and the row sums to the first
 // nm * S doubles of T: no step reads either before step A / T0 overwrite them.
-void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
-                         int nm, int S, float eps, int attempt, NewtonWork w, cudaStream_t s) {
+void launch_newton_bound_partial(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                                 int nm, int S, float eps, NewtonWork w, cudaStream_t s) {
   cudaMemsetAsync(w.T, 0, (size_t)nm * S * sizeof(double), s);
   newton_bound_partial_kernel<<<dim3((S + 31) / 32, nm), 256, 0, s>>>(A, a_stride, lda, upper, mats, S, eps,
                                                                       w.fro2, w.T);
+}
+
+void launch_newton_bound_final(const NewtonMat* mats, int nm, int S, float eps, int attempt, NewtonWork w,
+                               cudaStream_t s) {
   newton_bound_final_kernel<<<(nm + 7) / 8, 256, 0, s>>>(mats, nm, S, eps, attempt, w, w.T, w.T2);
+}
+
+void launch_newton_bound(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
+                         int nm, int S, float eps, int attempt, NewtonWork w, cudaStream_t s) {
+  launch_newton_bound_partial(A, a_stride, lda, upper, mats, nm, S, eps, w, s);
+  launch_newton_bound_final(mats, nm, S, eps, attempt, w, s);
 }
 
 void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, const NewtonMat* mats,
