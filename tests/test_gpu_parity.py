@@ -135,6 +135,17 @@ def test_block_128_many_tiles():
     assert_worst(w)
 
 
+@pytest.mark.parametrize("gdtype", ["f32", "bf16"])
+def test_block_1024_ragged_maximum_size(gdtype):
+    """The largest block side (b = 1024) with ragged last blocks in both
+    directions (1100 = 1024 + 76, 1030 = 1024 + 6) and a 1-D parameter longer
+    than one segment."""
+    shapes = [(1100, 1030), (1030,)]
+    w = run_pair(shapes, 1024, 0.999, 1e-6, 1, 0.0, 0.1, gdtype, steps=3, interval=2, seed=15,
+                 gstd=1e-3, check_every=False)
+    assert_worst(w)
+
+
 def test_transformer_layer_b512_full_size():
     """The Transformer-layer set at full size in the bench's launch
     configuration: 21 steps, roots at steps 1 and 21."""
@@ -148,7 +159,7 @@ def test_transformer_layer_b512_full_size():
 # --------------------------------------------------------------------------
 # the batched inverse-root kernel on its own
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("n", [64, 100, 192, 512])
+@pytest.mark.parametrize("n", [64, 100, 192, 512, 1000, 1024])
 @pytest.mark.parametrize("p", [2, 4])
 def test_batched_root_vs_oracle(n, p):
     from shampoo_second_order_b200 import batched_inverse_root
