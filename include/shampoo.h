@@ -323,10 +323,13 @@ void shampoo_destroy(shampoo_ctx* ctx);
  *          -1-k when the matrix gave up at iteration k.  On give-up X_i holds
  *          c^{-1} I (c^p = the starting eigenvalue bound).
  *  stream  caller-owned cudaStream_t.
- * Allocates its float64 work space (6 n x n per matrix in flight, at most
- * 2 GiB) with cudaMalloc and frees it before returning.  Synchronises while it
- * runs, like shampoo_compute_roots.  Returns SHAMPOO_ENOTCONVERGED if any
- * matrix gave up.
+ * Allocates its float64 work space (7 n' x n' doubles per matrix in flight,
+ * n' = n rounded up to 64, at most 2 GiB) in stream order on `stream` from a
+ * memory pool the library keeps per device, and frees it back to that pool
+ * before returning: the pool keeps the memory (it is not returned to the
+ * driver), so calls after the first allocate without the driver.
+ * Synchronises while it runs, like shampoo_compute_roots.  Returns
+ * SHAMPOO_ENOTCONVERGED if any matrix gave up.
  */
 shampoo_status shampoo_batched_inverse_root(const float* A, float* X, int batch,
                                             int n, int p, float eps, double tol,

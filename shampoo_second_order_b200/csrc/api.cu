@@ -184,6 +184,9 @@ struct shampoo_ctx {
   bool stats_done = false, roots_done = false;
   int last_not_converged = 0, last_max_iters = 0;
   int64_t generation = 0;            // root sets put in use so far
+  // the batched root call allocates from this stream-ordered pool (not owned)
+  cudaMemPool_t pool = nullptr;
+  cudaStream_t pool_stream = nullptr;
   std::vector<int32_t> root_iters;   // per matrix, last compute_roots (-1-k: gave up at k)
   Profiler prof;
   std::string err;
@@ -237,7 +240,8 @@ cudaError_t dalloc(shampoo_ctx* ctx, T** p, size_t count) {
   *p = nullptr;
   if (count == 0) return cudaSuccess;
   void* q = nullptr;
-  cudaError_t e = cudaMalloc(&q, count * sizeof(T));
+  cudaError_t e = ctx->pool ? cudaMallocFromPoolAsync(&q, count * sizeof(T), ctx->pool, ctx->pool_stream)
+                            : cudaMalloc(&q, count * sizeof(T));
   if (e == cudaSuccess) {
     ctx->allocs.push_back(q);
     *p = static_cast<T*>(q);
@@ -249,7 +253,11 @@ template <class T>
 shampoo_status upload(shampoo_ctx* ctx, T** dst, const std::vector<T>& v) {
   cudaError_t e = dalloc(ctx, dst, v.size());
   if (e != cudaSuccess) return fail(ctx, SHAMPOO_ENOMEM, "cudaMalloc of the block table failed");
-  if (!v.empty()) CK(cudaMemcpy(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice));
+  if (v.empty()) return SHAMPOO_OK;
+  if (ctx->pool)   // stream-ordered memory: copy in the allocation's stream (pageable source: staged before return)
+    CK(cudaMemcpyAsync(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice, ctx->pool_stream));
+  else
+    CK(cudaMemcpy(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice));
   return SHAMPOO_OK;
 }
 
@@ -490,6 +498,33 @@ shampoo_status ensure_ozaki(shampoo_ctx* ctx) {
   ctx->nw.qe = qe;
   ctx->nw.qcap = cap;
   return SHAMPOO_OK;
+}
+
+// A stream-ordered memory pool per device for shampoo_batched_inverse_root:
+// it keeps the memory its allocations return (release threshold: unlimited),
+// so a call after the first one allocates and frees its work space without
+// going back to the driver.
+cudaError_t batched_pool(cudaMemPool_t* out) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if ((e = cudaMemPoolCreate(&p, &props)) != cudaSuccess) return e;
+    uint64_t keep = UINT64_MAX;
+    if ((e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) return e;
+    pools[dev] = p;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
 }
 
 // ---------------- asynchronous root pipeline ----------------
@@ -1183,6 +1218,11 @@ shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int bat
   const bool use_oz = method == SHAMPOO_ROOTS_INT8_EMULATED;
   int kerr = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    const cudaError_t pe = batched_pool(&ctx->pool);
+    if (pe != cudaSuccess) return fail(nullptr, SHAMPOO_ECUDA, std::string("memory pool: ") + cudaGetErrorString(pe));
+    ctx->pool_stream = st;
+  }
   const int S = (n + kTile - 1) / kTile * kTile;
   const size_t per = 7 * (size_t)S * S * sizeof(double);
   const int chunk = (int)std::max<size_t>(1, std::min<size_t>(batch, (size_t(2) << 30) / per));
@@ -1232,9 +1272,9 @@ shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int bat
   }
   if (res == SHAMPOO_OK && nf) res = fail(ctx, SHAMPOO_ENOTCONVERGED, std::to_string(nf) + " roots did not converge");
 done:
-  cudaStreamSynchronize(st);
-  for (void* q : ctx->allocs) cudaFree(q);
+  for (void* q : ctx->allocs) cudaFreeAsync(q, st);   // back to the pool, in stream order
   ctx->allocs.clear();
+  cudaStreamSynchronize(st);
   if (ctx->h_count) cudaFreeHost(ctx->h_count);
   ctx->h_count = nullptr;
   for (auto& ev : ctx->ev)
