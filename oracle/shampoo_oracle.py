@@ -11,7 +11,7 @@ What it follows (all citations are to the pages on "Scalable Second Order
 Optimization for Deep Learning", Anil, Gupta, Koren, Regan, Singer):
 
 * arXiv abstract (mlsanity.com/paper/2002.09018, "Abstract"): the method is
-  a variant of full-matrix Adagrad.
+  a form of full-matrix Adagrad.
 * podcast transcript (podcast.do-not-panic.com, segments 6-8): Shampoo keeps
   one small matrix per dimension of a weight, L for the rows and R for the
   columns, and uses their Kronecker product in place of the full

@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
       be[j] = b;
     }
     kk = j + 1;
-    if (!(b > 1e-13 * fabs(a)) || !(b <= DBL_MAX)) break;   // invariant subspace (or garbage)
+    if (!(b > 1e-13 * fabs(a)) || !(b <= DBL_MAX)) break;   // invariant subspace (or a non-finite value)
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
       vp[i] = v[i];
       v[i] = wv[i] / b;
