@@ -754,7 +754,7 @@ def main():
                "copies": "pinned host; uploads and downloads on two copy streams, overlapped with compute"}
 
     # ---- asynchronous roots: the same K steps with the root job queued on the
-    # library's low-priority stream after step 0's statistics and swapped in by
+    # library's low-priority stream after step 0's statistics and installed by
     # a later apply; the region ends when the job has been installed ----
     async_line = None
     if not args.no_async:

@@ -137,7 +137,7 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx);
  * shampoo_compute_roots_async -- the same root computation, pipelined behind
  * the training steps (podcast transcript, segment 16: the statistics and the
  * preconditioned step keep running on the current roots while the next roots
- * are computed elsewhere, then swapped in; segment 14: roots a few steps old
+ * are computed elsewhere and take over once ready; segment 14: roots a few steps old
  * cost next to nothing in quality).
  *
  * Enqueues on the context's stream a copy of the statistics as they stand
