@@ -106,13 +106,14 @@ def apply_flops(cfg):
 
 def newton_flops(cfg, iters, per_kernel=False):
     """Symmetric products: n^2 (n+1) flops each (the upper triangle), times
-    products per step, times the iterations each matrix ran."""
+    products per step, times the iterations each matrix ran; the first step's
+    X0 T0 is a scaled copy (X0 = c^{-1} I), not a product."""
     sizes = matrix_sizes(cfg)
     a = b = c = 0
     for (n, prods), k in zip(sizes, iters):
         k = k if k >= 0 else -1 - k
         f = n * n * (n + 1)
-        a += 2 * k * f
+        a += (2 * k - (1 if k > 0 else 0)) * f
         b += (k * f) if prods == 4 else 0
         c += k * f
     return (a, b, c) if per_kernel else a + b + c
@@ -466,7 +467,8 @@ def roots_bench(args):
             for p, it in its:
                 k = it.cpu().numpy()
                 k = np.where(k >= 0, k, -1 - k)
-                flops += int(k.sum()) * (4 if p == 4 else 3) * n * n * (n + 1)
+                # the first step's X0 T0 is a scaled copy, not a product
+                flops += (int(k.sum()) * (4 if p == 4 else 3) - int((k > 0).sum())) * n * n * (n + 1)
     ms = sum(s.elapsed_time(e) for s, e in ev)
     val = flops / (ms * 1e-3) / 1e12
     line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": 1, "steps": args.steps,

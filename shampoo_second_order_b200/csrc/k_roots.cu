@@ -524,6 +524,20 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
   tri_tile(blockIdx.x, T, ti, tj);
   const size_t base = (size_t)m * S * S;
   const double* Tm = w.T + base;
+  if (blockIdx.z == 0 && it == 0) {
+    // X0 = c^{-1} I, so X1 = s_0^{1/p} c^{-1} T0 needs no product: the tile
+    // and its mirror (T0 is stored whole) are copied, scaled
+    const double sk = sched_at(w, m, 0);
+    const double sc = w.cinv[m] * (sk != 1.0 ? pow(sk, 1.0 / mats[m].p) : 1.0);
+    double* X1 = w.X[1] + base;
+    const int i0 = ti * TT, j0 = tj * TT;
+    for (int e = threadIdx.x; e < TT * TT; e += kNewtonThreads) {
+      const int a = e / TT, b = e % TT;
+      X1[(size_t)(i0 + a) * S + j0 + b] = sc * Tm[(size_t)(i0 + a) * S + j0 + b];
+      if (i0 != j0) X1[(size_t)(j0 + a) * S + i0 + b] = sc * Tm[(size_t)(j0 + a) * S + i0 + b];
+    }
+    return;
+  }
   const double* A = blockIdx.z == 0 ? w.X[it & 1] + base : Tm;
   double* C = blockIdx.z == 0 ? w.X[(it + 1) & 1] + base : w.T2 + base;
   double acc[FM][FM][2] = {};
