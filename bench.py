@@ -41,9 +41,10 @@ UNIT = "TFLOP/s"
 # ncu capture of the named kernel; None until measured for the current kernel.
 TRAFFIC_PER_LAUNCH = {
     # the 9 launches of the timed root step of the default Transformer-layer
-    # run (5 with every matrix iterating: ~1.01 GB each; 3 with a few: 17 MB;
-    # 1 with none), averaged like `achieved`
-    "newton_step_a": 566475065,
+    # run (the first, whose X product is a scaled copy: 0.80 GB; 4 more with
+    # every matrix iterating: ~1.01 GB each; 3 with a few: 17 MB; 1 with
+    # none), averaged like `achieved`
+    "newton_step_a": 542798336,
 }
 
 
