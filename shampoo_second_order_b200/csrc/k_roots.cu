@@ -319,8 +319,10 @@ __global__ void __launch_bounds__(256) newton_init_kernel(const float* __restric
 // ---------------------------------------------------------------------------
 constexpr int kLanczos = 12;
 
+// One scalar Newton step on an eigenvalue m of the scaled M: m ((p+1-m)/p)^p.
+// p is 2 or 4, so the division is a multiplication by the exact 1/p.
 __device__ __forceinline__ double newton_map(double m, int p) {
-  const double t = (p + 1 - m) / p;
+  const double t = (p + 1 - m) * (p == 4 ? 0.25 : 0.5);
   const double t2 = t * t;
   return m * (p == 4 ? t2 * t2 : t2);
 }
@@ -338,7 +340,27 @@ __device__ int sturm_count(const double* a, const double* b, int k, double x) {
   return cnt;
 }
 
-// Smallest (which = 1) or largest (which = k) eigenvalue of the tridiagonal.
+// Multisection over one warp: f is nondecreasing-true on [lo, hi] (false
+// below the point sought, true at and above it).  Each round the 32 lanes
+// test 32 evenly spaced interior points and the bracket shrinks 33-fold to
+// the cell where f turns true; every lane ends with the same bracket.
+template <class F>
+__device__ void warp_multisect(double& lo, double& hi, int rounds, F f) {
+  const int lane = threadIdx.x & 31;
+  for (int r = 0; r < rounds; ++r) {
+    const double h = (hi - lo) * (1.0 / 33.0);
+    const unsigned hit = __ballot_sync(0xffffffffu, f(lo + h * (lane + 1)));
+    const int j = hit ? __ffs(hit) - 1 : 32;   // first point where f holds
+    const double nlo = lo + h * j;
+    if (j < 32) hi = lo + h * (j + 1);
+    lo = nlo;
+  }
+}
+
+// Smallest (which = 1) or largest (which = k) eigenvalue of the tridiagonal:
+// Gershgorin bracket, then Sturm counts by warp multisection (12 rounds take
+// the bracket down by 33^12, below a double's resolution).  Called by a whole
+// warp.
 __device__ double tridiag_eig(const double* a, const double* b, int k, int which) {
   double lo = a[0], hi = a[0];
   for (int i = 0; i < k; ++i) {
@@ -346,11 +368,7 @@ __device__ double tridiag_eig(const double* a, const double* b, int k, int which
     lo = fmin(lo, a[i] - r);
     hi = fmax(hi, a[i] + r);
   }
-  for (int it = 0; it < 100; ++it) {
-    const double mid = 0.5 * (lo + hi);
-    if (sturm_count(a, b, k, mid) >= which) hi = mid;
-    else lo = mid;
-  }
+  warp_multisect(lo, hi, 12, [&](double x) { return sturm_count(a, b, k, x) >= which; });
   return 0.5 * (lo + hi);
 }
 
@@ -457,8 +475,9 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
     __syncthreads();
   }
   __syncthreads();
-  if (threadIdx.x != 0) return;
-  // interval estimate, kept inside what is guaranteed: [ridge / c^p, 1]
+  if (warp != 0) return;
+  // interval estimate, kept inside what is guaranteed: [ridge / c^p, 1]; the
+  // warp computes it together (the same values in every lane), lane 0 stores
   const double lo_g = w.ridge[m] / w.T2[m];   // T2 holds c^p until the first step
   double l = tridiag_eig(al, be, kk, 1), u = tridiag_eig(al, be, kk, kk);
   int ns = 0;
@@ -472,12 +491,8 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
       double a = 1.0 / u, b = fmin((p + 1) / u, cap), s;
       if (newton_map(b * l, p) <= newton_map(b * u, p)) {
         s = b;
-      } else {
-        for (int it = 0; it < 80; ++it) {
-          const double mid = 0.5 * (a + b);
-          if (newton_map(mid * l, p) < newton_map(mid * u, p)) a = mid;
-          else b = mid;
-        }
+      } else {   // 16 rounds: 33^16 > 2^80
+        warp_multisect(a, b, 16, [&](double x) { return !(newton_map(x * l, p) < newton_map(x * u, p)); });
         s = 0.5 * (a + b);
       }
       const double x = newton_map(s * l, p), y = newton_map(s * u, p);
@@ -485,10 +500,11 @@ __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __
       const double nu = (s * l <= 1.0 && s * u >= 1.0) ? 1.0 : fmax(x, y);
       l = nl;
       u = fmax(nu, nl);
-      sch[ns++] = s;
+      if (lane == 0) sch[ns] = s;
+      ++ns;
     }
   }
-  w.nsched[m] = ns;
+  if (lane == 0) w.nsched[m] = ns;
 }
 
 __device__ __forceinline__ double sched_at(const NewtonWork& w, int m, int k) { return newton_sched(w, m, k); }
