@@ -319,7 +319,7 @@ def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak, slices
         by = sets * S * S * (8 + slices)                              # read float64, write the slices
         work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")
     elif top == "newton_lanczos":
-        by = sum(12 * 8 * n * n for n, _ in matrix_sizes(cfg)) * n_root_steps
+        by = sum(12 * 4 * n * n for n, _ in matrix_sizes(cfg)) * n_root_steps   # 12 matvecs, fp32 operator
         work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / max(launches, 1), "MEASURED_PEAKS.json hbm_gbs")
     elif top == "update":
         by = el * (4 + 8 + (8 if cfg["momentum"] else 0)) * steps

@@ -278,7 +278,8 @@ cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
   if ((e = dalloc(ctx, &w.worse, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.iters, chunk)) != cudaSuccess) return e;
   if ((e = dalloc(ctx, &w.state, chunk)) != cudaSuccess) return e;
-  if ((e = dalloc(ctx, &w.count, 2)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.live, chunk)) != cudaSuccess) return e;
+  if ((e = dalloc(ctx, &w.count, 3)) != cudaSuccess) return e;
   return e;
 }
 
@@ -354,9 +355,11 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
           // under two CTAs per SM
           const int t64 = (S / 64) * (S / 64 + 1) / 2;
           const int tile = (int64_t)known * t64 * 2 <= 2 * 148 ? 32 : 64;
-          run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, nm, S, it, tile, w, st); });
-          if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, nm, S, tile, w, st); });
-          run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, nm, S, it, tile, w, st); });
+          // the grid covers `known` matrices; the check before this step
+          // listed the running ones (at most that many) in w.live
+          run(pr, "newton_step_a", st, [&] { launch_newton_step_a(d, known, S, it, tile, w, st); });
+          if (has_p4) run(pr, "newton_step_b", st, [&] { launch_newton_step_b(d, known, S, tile, w, st); });
+          run(pr, "newton_step_c", st, [&] { launch_newton_step_c(d, known, S, it, tile, w, st); });
         }
         run(pr, "newton_check", st, [&] { launch_newton_check(nm, it + 1, tol, max_iters, w, st); });
         const int nx = (it + 1) & 1;

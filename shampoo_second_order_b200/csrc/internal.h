@@ -99,11 +99,13 @@ struct NewtonWork {
   double* fro2;                 // [nmat] ||M-I||_F^2 of the valid corner
   double* prev;                 // [nmat] previous residual
   int* worse;                   // [nmat]
-  int* active;                  // [nmat]
+  int* live;                    // [nmat] the matrices the next step works on (running or
+                                //        X-only), in index order, listed by each check
   int* iters;                   // [nmat] iterations done
   int* state;                   // [nmat] 0 running, 1 converged, 2 failed, 3 diverged,
                                 //        4 one X-only step left
-  int* count;                   // [1] matrices still active after a check
+  int* count;                   // [3] matrices still active after check k: [k & 1] for the
+                                //     host to read back, [2] the length of `live`
   // int8 slices of the iterates for the emulated-float64 products (k_ozaki.cu):
   //   q   int8 [kOzSets][qs][qcap][S][S], slice k of set z for matrix m at
   //       plane (z * qs + k) * qcap + m
@@ -144,9 +146,12 @@ void launch_newton_t0(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaSt
 // one Newton step: A (X T and T T), B (T2 T2, p = 4 only), C (T^p M,
 // residual, next T) on tiles of side `tile` (64, or 32 when few matrices are
 // left); check k: convergence test of M_k
-void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s);
-void launch_newton_step_b(const NewtonMat* mats, int nm, int S, int tile, NewtonWork w, cudaStream_t s);
-void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s);
+// One Newton step over the matrices the last check listed in w.live; `rows`
+// (the grid's matrix extent) is any upper bound on their number, e.g. the
+// count a previous check reported.
+void launch_newton_step_a(const NewtonMat* mats, int rows, int S, int it, int tile, NewtonWork w, cudaStream_t s);
+void launch_newton_step_b(const NewtonMat* mats, int rows, int S, int tile, NewtonWork w, cudaStream_t s);
+void launch_newton_step_c(const NewtonMat* mats, int rows, int S, int it, int tile, NewtonWork w, cudaStream_t s);
 void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s);
 
 // ---------------- emulated float64 Newton products (k_ozaki.cu) ----------------

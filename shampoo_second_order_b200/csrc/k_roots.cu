@@ -532,7 +532,8 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
     const NewtonMat* __restrict__ mats, int S, int it, NewtonWork w) {
   constexpr int FM = TT / 16;
   __shared__ NewtonSmem<TT> sm;
-  const int m = blockIdx.y;
+  if ((int)blockIdx.y >= w.count[2]) return;   // the check listed fewer
+  const int m = w.live[blockIdx.y];
   const int st = w.state[m];
   if (st != kRunning && !(st == kFinal && blockIdx.z == 0)) return;
   const int T = S / TT;
@@ -579,7 +580,8 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_b_kernel(
     const NewtonMat* __restrict__ mats, int S, NewtonWork w) {
   constexpr int FM = TT / 16;
   __shared__ NewtonSmem<TT> sm;
-  const int m = blockIdx.y;
+  if ((int)blockIdx.y >= w.count[2]) return;   // the check listed fewer
+  const int m = w.live[blockIdx.y];
   if (w.state[m] != kRunning || mats[m].p != 4) return;
   const int T = S / TT;
   int ti, tj;
@@ -596,7 +598,8 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
   constexpr int FM = TT / 16, HALF = TT / 2;
   __shared__ NewtonSmem<TT> sm;
   __shared__ double red[kNewtonThreads / 32];
-  const int m = blockIdx.y;
+  if ((int)blockIdx.y >= w.count[2]) return;   // the check listed fewer
+  const int m = w.live[blockIdx.y];
   if (w.state[m] != kRunning) return;
   const int p = mats[m].p;
   const int T = S / TT;
@@ -651,47 +654,69 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_c_kernel(
 
 // Convergence test of M_k for every matrix (k = iterations done), in the
 // same order as the oracle: non-finite, tolerance, cap, 5 non-decreasing.
-__global__ void newton_check_kernel(int nm, int k, double tol, int max_iters, NewtonWork w) {
-  int alive = 0;
-  for (int m = threadIdx.x; m < nm; m += blockDim.x) {
-    if (w.state[m] == kFinal) {   // its last step computed X alone
-      w.state[m] = kConverged;
-      w.iters[m] = k;
-      continue;
+// The matrices the next step works on are listed in w.live in index order
+// (a ballot and a scan over the warps per 1024 matrices), their number in
+// w.count[2] and, for the host, in w.count[k & 1].  One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) newton_check_kernel(int nm, int k, double tol, int max_iters,
+                                                            NewtonWork w) {
+  __shared__ int wcount[32];
+  __shared__ int listed;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) listed = 0;
+  __syncthreads();
+  for (int m0 = 0; m0 < nm; m0 += blockDim.x) {
+    const int m = m0 + threadIdx.x;
+    bool keep = false;
+    if (m < nm) {
+      const int s0 = w.state[m];
+      if (s0 == kFinal) {   // its last step computed X alone
+        w.state[m] = kConverged;
+        w.iters[m] = k;
+      } else if (s0 == kRunning) {
+        const double r = __longlong_as_double(static_cast<long long>(w.resid[m]));
+        const double f = sqrt(w.fro2[m]);
+        w.resid[m] = 0ull;
+        w.fro2[m] = 0.0;
+        w.iters[m] = k;
+        // For a PSD A every eigenvalue of M stays in (0, 1], so max|M - I| < 1;
+        // a residual above 1.5 means rounding made A + ridge I indefinite.
+        int st = kRunning;
+        if (!(r <= 1.5)) {
+          st = kDiverged;
+        } else if (r <= tol) {
+          st = kConverged;
+        } else if (k >= max_iters) {
+          st = kFailed;
+        } else if (k >= w.nsched[m] && k > 0 && f <= 0.05 && 0.75 * f * f * (1.0 + f) <= 0.5 * tol) {
+          st = kFinal;   // one more step certainly lands below tol: compute X only
+        } else if (k >= w.nsched[m]) {   // the scaled steps may raise the residual
+          const int wo = (r >= w.prev[m]) ? w.worse[m] + 1 : 0;
+          w.worse[m] = wo;
+          w.prev[m] = r;
+          if (wo >= 5) st = kDiverged;
+        }
+        w.state[m] = st;
+        keep = (st == kRunning || st == kFinal);
+      }
     }
-    if (w.state[m] != kRunning) continue;
-    const double r = __longlong_as_double(static_cast<long long>(w.resid[m]));
-    const double f = sqrt(w.fro2[m]);
-    w.resid[m] = 0ull;
-    w.fro2[m] = 0.0;
-    w.iters[m] = k;
-    // For a PSD A every eigenvalue of M stays in (0, 1], so max|M - I| < 1;
-    // a residual above 1.5 means rounding made A + ridge I indefinite.
-    int st = kRunning;
-    if (!(r <= 1.5)) {
-      st = kDiverged;
-    } else if (r <= tol) {
-      st = kConverged;
-    } else if (k >= max_iters) {
-      st = kFailed;
-    } else if (k >= w.nsched[m] && k > 0 && f <= 0.05 && 0.75 * f * f * (1.0 + f) <= 0.5 * tol) {
-      st = kFinal;   // one more step certainly lands below tol: compute X only
-    } else if (k >= w.nsched[m]) {   // the scaled steps may raise the residual
-      const int wo = (r >= w.prev[m]) ? w.worse[m] + 1 : 0;
-      w.worse[m] = wo;
-      w.prev[m] = r;
-      if (wo >= 5) st = kDiverged;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) wcount[warp] = __popc(bal);
+    __syncthreads();
+    int pos = listed + __popc(bal & ((1u << lane) - 1u));
+    for (int q = 0; q < warp; ++q) pos += wcount[q];
+    if (keep) w.live[pos] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int q = 0; q < (int)(blockDim.x >> 5); ++q) t += wcount[q];
+      listed += t;
     }
-    w.state[m] = st;
-    alive += (st == kRunning || st == kFinal);
+    __syncthreads();
   }
-  // number of matrices still running (or with their X-only step left)
-  __shared__ int total;
-  if (threadIdx.x == 0) total = 0;
-  __syncthreads();
-  if (alive) atomicAdd(&total, alive);
-  __syncthreads();
-  if (threadIdx.x == 0) w.count[k & 1] = total;
+  if (threadIdx.x == 0) {
+    w.count[2] = listed;
+    w.count[k & 1] = listed;
+  }
 }
 
 __global__ void newton_reset_kernel(int nm, NewtonWork w) {
@@ -779,25 +804,28 @@ static int num_tri(int S, int tile) {
   return T * (T + 1) / 2;
 }
 
-void launch_newton_step_a(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
+void launch_newton_step_a(const NewtonMat* mats, int rows, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
+  if (rows < 1) return;
   if (tile == 32)
-    newton_step_a_kernel<32><<<dim3(num_tri(S, 32), nm, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+    newton_step_a_kernel<32><<<dim3(num_tri(S, 32), rows, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
   else
-    newton_step_a_kernel<64><<<dim3(num_tri(S, 64), nm, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+    newton_step_a_kernel<64><<<dim3(num_tri(S, 64), rows, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
 }
 
-void launch_newton_step_b(const NewtonMat* mats, int nm, int S, int tile, NewtonWork w, cudaStream_t s) {
+void launch_newton_step_b(const NewtonMat* mats, int rows, int S, int tile, NewtonWork w, cudaStream_t s) {
+  if (rows < 1) return;
   if (tile == 32)
-    newton_step_b_kernel<32><<<dim3(num_tri(S, 32), nm), kNewtonThreads, 0, s>>>(mats, S, w);
+    newton_step_b_kernel<32><<<dim3(num_tri(S, 32), rows), kNewtonThreads, 0, s>>>(mats, S, w);
   else
-    newton_step_b_kernel<64><<<dim3(num_tri(S, 64), nm), kNewtonThreads, 0, s>>>(mats, S, w);
+    newton_step_b_kernel<64><<<dim3(num_tri(S, 64), rows), kNewtonThreads, 0, s>>>(mats, S, w);
 }
 
-void launch_newton_step_c(const NewtonMat* mats, int nm, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
+void launch_newton_step_c(const NewtonMat* mats, int rows, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
+  if (rows < 1) return;
   if (tile == 32)
-    newton_step_c_kernel<32><<<dim3(num_tri(S, 32), nm), kNewtonThreads, 0, s>>>(mats, S, it, w);
+    newton_step_c_kernel<32><<<dim3(num_tri(S, 32), rows), kNewtonThreads, 0, s>>>(mats, S, it, w);
   else
-    newton_step_c_kernel<64><<<dim3(num_tri(S, 64), nm), kNewtonThreads, 0, s>>>(mats, S, it, w);
+    newton_step_c_kernel<64><<<dim3(num_tri(S, 64), rows), kNewtonThreads, 0, s>>>(mats, S, it, w);
 }
 
 void launch_newton_check(int nm, int k, double tol, int max_iters, NewtonWork w, cudaStream_t s) {

@@ -93,10 +93,10 @@ size_t carve(unsigned char* base, int chunk, int S, NewtonWork* w, NewtonMat** m
   w->fro2 = c.take<double>(chunk);
   w->prev = c.take<double>(chunk);
   w->worse = c.take<int>(chunk);
-  w->active = nullptr;
+  w->live = c.take<int>(chunk);
   w->iters = c.take<int>(chunk);
   w->state = c.take<int>(chunk);
-  w->count = c.take<int>(2);
+  w->count = c.take<int>(3);
   *mats = c.take<NewtonMat>(chunk);
   *retry = c.take<NewtonMat>(chunk);
   *nretry = c.take<int>(1);
@@ -196,9 +196,9 @@ extern "C" shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, f
       int alive = 0;
       e = read_int(&w.count[0], &alive, st);
       for (int it = 0; it < max_iters && alive && e == cudaSuccess; ++it) {
-        launch_newton_step_a(mats, nm, S, it, 64, w, st);
-        if (p == 4) launch_newton_step_b(mats, nm, S, 64, w, st);
-        launch_newton_step_c(mats, nm, S, it, 64, w, st);
+        launch_newton_step_a(mats, alive, S, it, 64, w, st);   // `alive`: the last check's count
+        if (p == 4) launch_newton_step_b(mats, alive, S, 64, w, st);
+        launch_newton_step_c(mats, alive, S, it, 64, w, st);
         launch_newton_check(nm, it + 1, tol, max_iters, w, st);
         e = read_int(&w.count[(it + 1) & 1], &alive, st);
       }
