@@ -375,7 +375,7 @@ __device__ double tridiag_eig(const double* a, const double* b, int k, int which
 // One CTA per matrix: kLanczos Lanczos steps on the valid corner of M0
 // (float64 vectors, the float32 statistic as the operator; no
 // reorthogonalisation: only the extreme Ritz values are used),
-// their extreme eigenvalues by Sturm bisection, and the schedule s_k.
+// their extreme eigenvalues by Sturm multisection, and the schedule s_k (both on warp 0).
 __global__ void __launch_bounds__(512) newton_lanczos_kernel(const NewtonMat* __restrict__ mats, int S,
                                                              NewtonWork w) {
   __shared__ double v[1024], vp[1024], wv[1024];
