@@ -96,6 +96,28 @@ def test_newton_agrees_with_eigh(p, kappa):
     assert np.linalg.norm(X - ref) / np.linalg.norm(ref) < 1e-9
 
 
+def _denman_beavers(B, iters=60):
+    """Square root and inverse square root of an SPD matrix by the
+    Denman-Beavers iteration (Y <- (Y + Z^{-1})/2, Z <- (Z + Y^{-1})/2 from
+    Y = B, Z = I), a third route that shares nothing with eigh or Newton."""
+    Y, Z = B.copy(), np.eye(B.shape[0])
+    for _ in range(iters):
+        Y, Z = 0.5 * (Y + np.linalg.inv(Z)), 0.5 * (Z + np.linalg.inv(Y))
+    return Y, Z
+
+
+@pytest.mark.parametrize("p", [2, 4])
+def test_root_matches_denman_beavers(p):
+    """(A + eps I)^{-1/2} is Denman-Beavers' Z; (A + eps I)^{-1/4} is the
+    inverse square root of its square root Y."""
+    A, _ = rand_spd(16, 1e4, seed=21 + p)
+    B = A + 1e-6 * np.eye(16)
+    Y, Z = _denman_beavers(B)
+    ref = Z if p == 2 else _denman_beavers(Y)[1]
+    X = inverse_root(A, 1e-6, p)
+    assert np.linalg.norm(X - ref) / np.linalg.norm(ref) < 1e-10
+
+
 def test_newton_tolerance_1e6_is_enough_for_1e3():
     """At the cfg tolerance (max|M-I| <= 1e-6) Newton is far inside 1e-3."""
     A, _ = rand_spd(48, 1e8, 21)
