@@ -38,13 +38,15 @@ METRIC = "Shampoo optimizer step ms and TFLOP/s (stats+roots+apply) vs B200 peak
 UNIT = "TFLOP/s"
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
-# ncu capture of the named kernel; None until measured for the current kernel.
+# ncu capture of the named kernel on the named workload (float64 Newton
+# products, both factors, the default --steps/--warmup); None for any other
+# workload, mode or kernel until measured there.
 TRAFFIC_PER_LAUNCH = {
-    # the 9 launches of the timed root step of the default Transformer-layer
-    # run (the first, whose X product is a scaled copy: 0.80 GB; 4 more with
-    # every matrix iterating: ~1.01 GB each; 3 with a few: 17 MB; 1 with
-    # none), averaged like `achieved`
-    "newton_step_a": 542061340,
+    # the 9 launches of the timed root step of the Transformer-layer run (the
+    # first, whose X product is a scaled copy: 0.80 GB; 4 more with every
+    # matrix iterating: ~1.01 GB each; 3 with a few: 17 MB; 1 with none),
+    # averaged like `achieved`
+    ("transformer_layer_b512", "newton_step_a"): 542061340,
 }
 
 
@@ -277,7 +279,7 @@ def tc_work(cfg, kernel):
     return fl, by
 
 
-def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak, slices=6):
+def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak, slices=6, traffic_key=None):
     """Achieved vs peak for the kernel with the largest share of device time."""
     names = {k: v for k, v in prof.items() if v[1] > 0}
     if not names:
@@ -332,7 +334,7 @@ def roofline(cfg, prof, iters_sum, steps, n_root_steps, peaks, fp64_peak, slices
     if work is None:
         return top, None
     bound, ach, peak, unit, per_launch, src = work
-    tr = TRAFFIC_PER_LAUNCH.get(top)
+    tr = TRAFFIC_PER_LAUNCH.get((traffic_key, top)) if traffic_key else None
     return top, {"kernel": top, "bound": bound, "achieved": round(ach, 3), "peak": round(peak, 2),
                  "unit": unit, "frac": round(ach / peak, 4), "traffic": tr,
                  "algorithmic_per_launch": per_launch, "launches": launches,
@@ -797,7 +799,9 @@ def main():
                       "sync_step_ms_max": max(s_.elapsed_time(e_) for s_, e_ in ev),
                       "streams": "steps at high priority; roots on the library's lowest-priority stream"}
 
-    top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak, args.slices)
+    # the committed DRAM traffic holds only for the workload and mode it was captured on
+    tkey = args.config if (args.roots == "fp64" and not args.one_sided_embedding) else None
+    top, roof = roofline(cfg, prof, iters_sum, args.steps, n_root, peaks, fp64_peak, args.slices, tkey)
 
     if rank == 0:
         phase = {}

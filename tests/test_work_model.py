@@ -75,3 +75,21 @@ def test_one_sided_blocks_drop_a_factor():
 def test_job_throughput_is_total_work_over_the_slowest_rank():
     # 1e12 flops per rank on 4 ranks in 2 ms: 2000 TFLOP/s for the job
     assert abs(bench.job_tflops(1e12, 4, 2.0) - 2000.0) < 1e-9
+
+
+def test_committed_dram_traffic_is_reported_only_for_its_workload():
+    """The ncu traffic per launch was captured on one workload; the roofline
+    block carries it there and null everywhere else."""
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}
+    for name, key, expect in [("transformer_layer_b512", "transformer_layer_b512", True),
+                              ("transformer_big_b1024", "transformer_big_b1024", False),
+                              ("transformer_layer_b512", None, False)]:
+        c = wl.CONFIGS[name]
+        n = len(bench.matrix_sizes(c))
+        prof = {"newton_step_a": (9, 5.0), "stats_tc": (20, 1.0)}
+        top, roof = bench.roofline(c, prof, [7] * n, 20, 1, peaks, 35.0, 6, key)
+        assert top == "newton_step_a" and roof["bound"] == "tensor"
+        assert (roof["traffic"] is not None) == expect
+        # achieved = the launches' credited products over their event time
+        a = bench.newton_flops(c, [7] * n, per_kernel=True)[0]
+        assert abs(roof["achieved"] - a / 5e-3 / 1e12) < 1e-3 * roof["achieved"]
