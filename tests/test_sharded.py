@@ -1,6 +1,6 @@
 """Block-sharded data parallelism (segment 16, Lemma 2) on CPU: the owner
 plan from the C library, and the reduce-scatter / owner step / all-gather
-plumbing of ShardedShampoo over gloo with world size 2.
+plumbing of ShardedShampoo over gloo with world sizes 2 and 3.
 
 The ranks' local optimizer here is the fp64 oracle on CPU tensors (the CUDA
 library needs a GPU); what is under test is the plumbing around it: after
@@ -131,8 +131,8 @@ def _worker(rank, world, port, q):
     q.put((rank, worst, same, opt.mine, opt.collective_bytes_per_step()))
 
 
-def test_sharded_step_matches_one_oracle_on_mean_gradients():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_step_matches_one_oracle_on_mean_gradients(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
