@@ -117,3 +117,53 @@ def test_package_import_does_not_load_library():
     importlib.reload(pkg)
     from shampoo_second_order_b200 import workloads  # noqa: F401
     assert hasattr(pkg, "lib")
+
+
+def _c_decls():
+    """(return type, name, [parameter types]) of every declaration in include/*.h."""
+    out = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for ret, name, args in re.findall(r"([A-Za-z_][\w\s\*]*?)\b(shampoo_\w+)\s*\(([^;{]*?)\)\s*;", text,
+                                          flags=re.S):
+            params = [] if args.strip() in ("", "void") else [" ".join(a.split()) for a in args.split(",")]
+            # drop the parameter name: the type is everything before the last identifier
+            types = [re.sub(r"\s*\b\w+$", "", p).replace(" *", "*") for p in params]
+            out.append((" ".join(ret.split()), name, types))
+    return out
+
+
+_SCALAR = {"int": C.c_int, "shampoo_graft": C.c_int, "shampoo_dtype": C.c_int, "int64_t": C.c_int64,
+           "int32_t": C.c_int32, "float": C.c_float, "double": C.c_double}
+
+
+def _matches(ctype, py):
+    t = re.sub(r"\bconst\b", "", ctype).replace(" ", "")
+    if t.endswith("*"):
+        pointee = t[:-1]
+        if pointee == "char":
+            return py in (C.c_char_p, C.c_void_p)
+        if py is C.c_void_p:   # an opaque or untyped pointer
+            return True
+        base = getattr(py, "_type_", None)
+        return base is not None and (_SCALAR.get(pointee) is base or pointee.endswith("*"))
+    return _SCALAR.get(t) is py
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature in the binding has the header's parameter count
+    and compatible types, so the binding cannot drift from the C-ABI."""
+    decls = _c_decls()
+    assert {n for _, n, _ in decls} == set(L.SIGNATURES)
+    rets = {"shampoo_status": C.c_int, "int": C.c_int, "int64_t": C.c_int64, "const char*": C.c_char_p,
+            "void": None}
+    for ret, name, types in decls:
+        res, args = L.SIGNATURES[name]
+        assert rets[re.sub(r"\s*\*", "*", ret)] is res, (name, ret, res)
+        assert len(types) == len(args), (name, types, args)
+        for t, a in zip(types, args):
+            assert _matches(t, a), (name, t, a)
