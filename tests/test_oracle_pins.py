@@ -96,6 +96,35 @@ def test_newton_agrees_with_eigh(p, kappa):
     assert np.linalg.norm(X - ref) / np.linalg.norm(ref) < 1e-9
 
 
+def _scalar_newton(lam, eps, p, tol=1e-6, max_iter=100):
+    """The coupled iteration on a diagonal matrix is one scalar iteration per
+    eigenvalue: m <- m ((p+1-m)/p)^p, x <- x (p+1-m)/p from m0 = (l+eps)/c^p,
+    x0 = c^{-1}, c^p = the largest l + eps (the max row sum of a diagonal)."""
+    lam = np.asarray(lam, dtype=np.float64) + eps
+    cp = lam.max()
+    m, x = lam / cp, np.full(lam.shape, cp ** (-1.0 / p))
+    for k in range(max_iter + 1):
+        if np.abs(m - 1.0).max() <= tol:
+            return x, k
+        t = (p + 1 - m) / p
+        x, m = x * t, t ** p * m
+    return x, None
+
+
+@pytest.mark.parametrize("p,counts", [(4, [9, 14, 19, 25]), (2, [10, 15, 21, 27])])
+def test_newton_on_a_diagonal_is_scalar_newton(p, counts):
+    """Iteration count and result of the matrix iteration equal those of the
+    scalar recurrence, over spectra spanning kappa = 1e2 ... 1e8 (the counts
+    grow by about 5 per factor of 100 in kappa, as the scalar map predicts)."""
+    for kappa, expect in zip([1e2, 1e4, 1e6, 1e8], counts):
+        lam = np.array([1.0, np.sqrt(kappa), kappa])
+        X, it, ok = coupled_newton_inverse_root(np.diag(lam), 1e-12, p)
+        xs, ks = _scalar_newton(lam, 1e-12, p)
+        assert ok and it == ks == expect, (kappa, it, ks)
+        assert np.allclose(np.diag(X), xs, rtol=1e-14, atol=0)
+        assert np.abs(X - np.diag(np.diag(X))).max() == 0.0
+
+
 def _denman_beavers(B, iters=60):
     """Square root and inverse square root of an SPD matrix by the
     Denman-Beavers iteration (Y <- (Y + Z^{-1})/2, Z <- (Z + Y^{-1})/2 from
