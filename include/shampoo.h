@@ -367,10 +367,12 @@ shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int bat
  * Any batch size is accepted; matrices are processed in chunks that fit the
  * work space (7 n' x n' doubles each, n' = n rounded up to 64).
  * Sharing: every call uses the same work space, so calls that overlap on the
- * GPU (from other streams or host threads) race; serialise them.  The first
- * call on a device looks up the work space's device address with that device
- * current; make that first call before any stream capture.  Synchronises
- * with the host while it runs.
+ * GPU (from other streams or host threads) race; serialise them.  Every call
+ * looks up the work space's device address on the current device (nothing is
+ * kept between calls, so a device reset cannot leave a stale address); the
+ * first lookup in a process may load the library's device code, so make the
+ * first call before any stream capture begins.  Synchronises with the host
+ * while it runs.
  */
 shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, float* X, int batch, int n,
                                                     int p, float eps, double tol, int max_iters,
@@ -412,6 +414,23 @@ shampoo_status shampoo_plan_shards(int nparams, const int64_t* shapes,
  * stream: caller-owned cudaStream_t.  Allocates and frees 4 bytes.
  */
 shampoo_status shampoo_selftest_stalled_wait(void* stream);
+
+/*
+ * shampoo_selftest_stall_next_stats -- failure-path check inside the product
+ * kernels: the next shampoo_update_stats of `ctx` launches its statistics
+ * GEMM with the MMA issuer first waiting, through the pipelines' bounded
+ * wait, on a barrier phase that nothing completes.  That wait runs out (about
+ * a second) exactly as a stalled pipeline would: the launch aborts, lets the
+ * loads it has in flight land, frees its tensor memory, sets the context's
+ * error word and returns.  update_stats itself returns SHAMPOO_OK (it does not
+ * wait for its kernels); the next call that synchronises --
+ * shampoo_compute_roots, shampoo_install_roots with wait, shampoo_root_status,
+ * shampoo_nonfinite_status -- returns SHAMPOO_ECUDA, and so does every step
+ * call after an apply has copied the error word back.  The context's
+ * statistics are then half-updated: destroy it.  A test of the error path:
+ * no fault, no hang.  SHAMPOO_EINVAL if ctx is NULL.
+ */
+shampoo_status shampoo_selftest_stall_next_stats(shampoo_ctx* ctx);
 
 /* Library version, "MAJOR.MINOR.PATCH". */
 const char* shampoo_version(void);

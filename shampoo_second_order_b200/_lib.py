@@ -53,6 +53,7 @@ SIGNATURES = {
     "shampoo_plan_shards": (C.c_int, [C.c_int, C.POINTER(C.c_int64), C.POINTER(C.c_int32), C.c_int, C.c_int,
                                       C.c_int, C.POINTER(C.c_int32), C.POINTER(C.c_double)]),
     "shampoo_selftest_stalled_wait": (C.c_int, [_P]),
+    "shampoo_selftest_stall_next_stats": (C.c_int, [_P]),
     "shampoo_version": (C.c_char_p, []),
 }
 
@@ -248,6 +249,10 @@ def shampoo_plan_shards(shapes, block_size, root_interval, nranks):
     cost = (C.c_double * int(nranks))()
     _check(lib().shampoo_plan_shards(n, dims, nd, int(block_size), int(root_interval), int(nranks), owner, cost))
     return list(owner), list(cost)
+
+
+def shampoo_selftest_stall_next_stats(ctx):
+    return _check(lib().shampoo_selftest_stall_next_stats(ctx), ctx)
 
 
 def shampoo_version():

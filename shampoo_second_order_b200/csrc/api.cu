@@ -177,7 +177,8 @@ struct shampoo_ctx {
   int root_method = SHAMPOO_ROOTS_FP64;   // or SHAMPOO_ROOTS_INT8_EMULATED
   int oz_slices = 6;
   OzakiMaps oz{};                          // over nw.q, once allocated
-  int* h_count = nullptr;   // pinned [2]
+  int* h_count = nullptr;   // pinned [3]: Newton counts [0..1], a copy of the error word [2]
+  int stall_next_stats = 0;  // failure-path test: the next statistics GEMM stalls and aborts
   cudaEvent_t ev[2] = {nullptr, nullptr};
   std::vector<void*> allocs;
 
@@ -283,16 +284,11 @@ cudaError_t alloc_newton(shampoo_ctx* ctx, NewtonWork& w, int chunk, int S) {
   return e;
 }
 
-// Run the Newton iteration over mats[0..nm) (device array dm) in chunks of
-// `chunk` matrices.  A/X are float32 slot arrays.  Returns the number of
-// matrices that gave up and the largest iteration count through outs.
 // Run the Newton iteration over the matrices hm (device copy dm) in chunks of
 // `chunk`.  A matrix whose iteration diverges (rounding left A + eps I
-// indefinite) is run again with the ridge raised, up to kAttempts times.
+// indefinite) is run again with the ridge raised, up to kNewtonAttempts times.
 // Reports the number of matrices that gave up, the largest iteration count
 // and, per matrix slot, the iterations (-1-k when it gave up at k).
-constexpr int kAttempts = 4;
-
 shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<NewtonMat>& hm,
                           const NewtonMat* dm, NewtonMat* d_retry, const float* A,
                           int64_t a_stride, int lda, int upper, float* X, int64_t x_stride, int ldx, int S,
@@ -312,7 +308,7 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
     std::vector<NewtonMat> list(hm.begin() + c0, hm.begin() + std::min(nm_all, c0 + chunk));
     const NewtonMat* d = dm + c0;
     std::vector<int> done_iters(list.size(), 0);
-    for (int attempt = 0; attempt < kAttempts && !list.empty(); ++attempt) {
+    for (int attempt = 0; attempt < kNewtonAttempts && !list.empty(); ++attempt) {
       const int nm = (int)list.size();
       int has_p4 = 0;
       for (const auto& m : list) has_p4 |= (m.p == 4);
@@ -376,7 +372,7 @@ shampoo_status run_newton(shampoo_ctx* ctx, Profiler* pr, const std::vector<Newt
       std::vector<NewtonMat> again;
       for (int i = 0; i < nm; ++i)
         if (hstate[i] == 3) again.push_back(list[i]);
-      const int final_pass = (attempt == kAttempts - 1) || again.empty();
+      const int final_pass = (attempt == kNewtonAttempts - 1) || again.empty();
       run(pr, "newton_finalize", st, [&] {
         launch_newton_finalize(X, x_stride, ldx, d, nm, S, w, has_root, iters_out, final_pass, st);
       });
@@ -446,12 +442,29 @@ bool encode_planes(CUtensorMap* m, void* base, int S, int64_t depth, int box_x, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A kernel that gave up on a wait leaves a code in the error word.
+constexpr const char* kTimeoutMsg =
+    "a tensor-core kernel timed out waiting on its pipeline and aborted; the optimizer state of this "
+    "context is no longer valid (destroy it and start a new one)";
+
+// A kernel that gave up on a wait leaves a code in the error word; the word
+// is never cleared, so once set every later check reports it.
 shampoo_status check_kernel_error(shampoo_ctx* ctx) {
   int e = 0;
   CK(cudaMemcpyAsync(&e, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost, ctx->stream));
   CK(cudaStreamSynchronize(ctx->stream));
-  if (e) return fail(ctx, SHAMPOO_ECUDA, "a tensor-core kernel timed out waiting on its pipeline");
+  if (e) {
+    if (ctx->h_count) ctx->h_count[2] = e;   // later polls refuse at once
+    return fail(ctx, SHAMPOO_ECUDA, kTimeoutMsg);
+  }
+  return SHAMPOO_OK;
+}
+
+// Non-blocking check at the start of a step call: every apply leaves a copy of
+// the error word in pinned host memory (copied in stream order after its
+// kernels), so a time-out of an earlier step is seen without waiting.
+shampoo_status poll_kernel_error(shampoo_ctx* ctx) {
+  if (ctx->h_count && *reinterpret_cast<volatile int*>(&ctx->h_count[2]))
+    return fail(ctx, SHAMPOO_ECUDA, kTimeoutMsg);
   return SHAMPOO_OK;
 }
 
@@ -596,6 +609,10 @@ shampoo_status install_roots(shampoo_ctx* ctx, bool wait, int* installed) {
   std::unique_lock<std::mutex> lock(ctx->job_mu);
   if (wait)
     ctx->cv.wait(lock, [&] { return ctx->job != shampoo_ctx::kQueued && ctx->job != shampoo_ctx::kRunning; });
+  if (wait) {   // a waiting install synchronises anyway: read the error word itself
+    const shampoo_status ks = check_kernel_error(ctx);
+    if (ks != SHAMPOO_OK) return ks;
+  }
   if (ctx->job != shampoo_ctx::kDone) return SHAMPOO_OK;
   ctx->job = shampoo_ctx::kIdle;
   const shampoo_status r = ctx->job_status;
@@ -815,7 +832,8 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
     shampoo_destroy(ctx);
     return fail(nullptr, SHAMPOO_ENOMEM, std::string("device allocation failed: ") + cudaGetErrorString(e));
   }
-  e = cudaMallocHost(&ctx->h_count, 2 * sizeof(int));
+  e = cudaMallocHost(&ctx->h_count, 3 * sizeof(int));
+  if (e == cudaSuccess) ctx->h_count[2] = 0;
   int prio = 0;
   if (e == cudaSuccess) e = cudaStreamGetPriority(ctx->stream, &prio);
   if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&ctx->aux, cudaStreamNonBlocking, prio);
@@ -856,7 +874,9 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
 
 shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
-  shampoo_status st = set_pointers(ctx, grads, nullptr);
+  shampoo_status st = poll_kernel_error(ctx);
+  if (st != SHAMPOO_OK) return st;
+  st = set_pointers(ctx, grads, nullptr);
   if (st != SHAMPOO_OK) return st;
   cudaStream_t s = ctx->stream, x = ctx->aux;
   const int nch = (int)ctx->chunks.size();
@@ -898,8 +918,9 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
     cudaError_t e = cudaSuccess;
     run(pr, "stats_tc", s, [&] {
       e = launch_stats_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S,
-                          ctx->planes_g, ctx->beta2, ctx->stats, ctx->d_err, s);
+                          ctx->planes_g, ctx->beta2, ctx->stats, ctx->d_err, s, ctx->stall_next_stats);
     });
+    ctx->stall_next_stats = 0;
     if (e != cudaSuccess) return cuda_fail(ctx, e, "stats_tc");
   }
   CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
@@ -913,6 +934,10 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
   int nf = 0, mi = 0;
   if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots before update_stats");
   if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "an asynchronous root job is in flight");
+  {   // statistics left by an aborted GEMM are not rooted: this call synchronises anyway
+    const shampoo_status ks = check_kernel_error(ctx);
+    if (ks != SHAMPOO_OK) return ks;
+  }
   {   // a finished job's roots are older than these: install, then overwrite
     const shampoo_status ir = install_roots(ctx, false, nullptr);
     if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
@@ -936,6 +961,10 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
     e = launch_split(ctx->roots, (int64_t)ctx->nmat * slot, ctx->rplanes, ctx->stream);
   });
   if (e != cudaSuccess) return cuda_fail(ctx, e, "split_roots");
+  {   // the emulated products' tensor-core kernels report time-outs here too
+    const shampoo_status ks = check_kernel_error(ctx);
+    if (ks != SHAMPOO_OK) return ks;
+  }
   ctx->roots_done = true;
   ++ctx->generation;
   ctx->last_not_converged = nf;
@@ -947,6 +976,10 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
 shampoo_status shampoo_compute_roots_async(shampoo_ctx* ctx) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots_async before update_stats");
+  {
+    const shampoo_status ks = poll_kernel_error(ctx);
+    if (ks != SHAMPOO_OK) return ks;
+  }
   if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "the previous asynchronous root job is still running");
   const shampoo_status ir = install_roots(ctx, false, nullptr);
   if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
@@ -985,6 +1018,10 @@ int64_t shampoo_roots_generation(const shampoo_ctx* ctx) { return ctx ? ctx->gen
 shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void* const* grads,
                              float lr) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  {
+    const shampoo_status ks = poll_kernel_error(ctx);
+    if (ks != SHAMPOO_OK) return ks;
+  }
   {
     const shampoo_status ir = install_roots(ctx, false, nullptr);
     if (ir != SHAMPOO_OK && ir != SHAMPOO_ENOTCONVERGED) return ir;
@@ -1039,6 +1076,8 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
                   ctx->p2, ctx->graft, ctx->mu, lr, ctx->mom, s);
   });
   CK(cudaGetLastError());
+  // the error word as it stands after this step, for the next call's poll
+  CK(cudaMemcpyAsync(&ctx->h_count[2], ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
   return SHAMPOO_OK;
 }
 
@@ -1122,6 +1161,12 @@ shampoo_status shampoo_set_one_sided(shampoo_ctx* ctx, int param, int side) {
                   cudaMemcpyHostToDevice));
   CK(launch_split(ctx->roots, (int64_t)ctx->nmat * S * S, ctx->rplanes, ctx->stream));
   CK(cudaStreamSynchronize(ctx->stream));
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_selftest_stall_next_stats(shampoo_ctx* ctx) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  ctx->stall_next_stats = 1;
   return SHAMPOO_OK;
 }
 
@@ -1246,7 +1291,7 @@ shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int bat
     res = fail(ctx, SHAMPOO_ENOMEM, std::string("work space: ") + cudaGetErrorString(e));
     goto done;
   }
-  if ((e = cudaMallocHost(&ctx->h_count, 2 * sizeof(int))) != cudaSuccess ||
+  if ((e = cudaMallocHost(&ctx->h_count, 3 * sizeof(int))) != cudaSuccess ||
       (e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming)) != cudaSuccess ||
       (e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming)) != cudaSuccess ||
       (e = dalloc(ctx, &ctx->d_err, 1)) != cudaSuccess ||

@@ -38,6 +38,10 @@ struct ParamDesc {
 constexpr int kChunk = 16384;   // elements per elementwise chunk
 constexpr int kSched = 32;      // longest Newton scaling schedule
 constexpr int kTile = 64;       // tile side of every matrix kernel
+// Newton runs per matrix: the first with the ridge eps, then up to three more
+// with the ridge raised after a divergence (both batched-root entry points
+// and the optimizer's root step).
+constexpr int kNewtonAttempts = 4;
 
 // Per-matrix bookkeeping of the Newton root iteration.
 struct NewtonMat {
@@ -64,9 +68,11 @@ cudaError_t launch_gather(const BlockDesc* blocks, int nblk, const void* const* 
 cudaError_t launch_split(const float* x, int64_t n, uint16_t* out, cudaStream_t s);
 // a wait that runs out: sets *err to the timeout code after about a second
 cudaError_t launch_stalled_wait(int* err, cudaStream_t s);
+// stall != 0 (failure-path test only): the MMA issuer first waits on a
+// barrier phase that nothing completes, runs out and aborts the launch
 cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
                             int nmat, int S, int planes_g, float beta2, float* stats, int* err,
-                            cudaStream_t s);
+                            cudaStream_t s, int stall = 0);
 cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
                               int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s);
 cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const ParamDesc* params,

@@ -48,6 +48,7 @@ struct TcArgs {
   float* P;          // parameter-shaped preconditioned gradient
   double* p2;        // [nparams] sum of P^2
   int* err;
+  int stall;         // failure-path test: the MMA issuer first waits on a phase nothing completes
 };
 
 __device__ __forceinline__ void tri_tile128(int idx, int T, int& ti, int& tj) {
@@ -154,7 +155,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   uint64_t* drain = tempty + 2;
   uint64_t* cfull = drain + 1;      // statistics tile loaded
   uint64_t* cready = cfull + 1;     // all epilogue threads wrote the tile (count 128)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cready + 1);
+  uint64_t* never = cready + 1;     // no thread ever arrives here (the failure-path test)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (tid == 0) {
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     tc::mbar_init(drain, 1);
     tc::mbar_init(cfull, 1);
     tc::mbar_init(cready, 128);
+    tc::mbar_init(never, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -231,8 +234,19 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         }
       }
     }
+    // Every load issued lands before the CTA retires: after an abort the MMA
+    // issuer no longer consumes the ring, so the last use of each stage may
+    // still be in flight.  (On the normal path these phases completed long
+    // ago and each wait returns at once.)
+    for (int q = g > ST ? g - ST : 0; q < g; ++q) tc::mbar_wait(&full[q % ST], (q / ST) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
+    // failure-path test: a bounded wait on a phase that nothing completes
+    // runs out exactly like a stalled pipeline and takes the abort path
+    if (args.stall && !tc::mbar_wait(never, 0)) {
+      *abort_flag = 1;
+      atomicExch(args.err, tc::kErrTimeout);
+    }
     int g = 0, i = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       const TileInfo x = decode_tile<MODE>(t, args);
@@ -627,11 +641,11 @@ cudaError_t launch_split(const float* x, int64_t n, uint16_t* out, cudaStream_t 
 
 cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
                             int nmat, int S, int planes_g, float beta2, float* stats, int* err,
-                            cudaStream_t s) {
+                            cudaStream_t s, int stall) {
   if (nblk <= 0) return cudaSuccess;
   TcArgs a{};
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
-  a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err;
+  a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err; a.stall = stall;
   const int T = (S + kTM - 1) / kTM;
   return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, planes_g, planes_g == 1),
                              maps, a, s);

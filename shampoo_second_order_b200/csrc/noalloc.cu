@@ -18,10 +18,12 @@
 //    buffers per matrix, n' = n rounded up to 64, so n <= 1024;
 //  * every call shares the array; calls that overlap on the GPU (other streams,
 //    other host threads) race and must be serialised by the caller;
-//  * the first call on a device looks up the array's device address there
-//    (cudaGetSymbolAddress with that device current); make that first call
-//    before any stream capture.
-#include <mutex>
+//  * every call looks up the array's device address on the current device
+//    (cudaGetSymbolAddress with that device current) instead of keeping it:
+//    after a device reset, or under another driver context, the array can sit
+//    at another address, and a kept one would point at freed memory.  The
+//    first lookup in a process may load the library's device code, so make
+//    the first call before any stream capture begins.
 #include <string>
 
 #include "../../include/shampoo.h"
@@ -34,31 +36,16 @@ void set_global_error(const std::string& msg);   // api.cu
 namespace {
 
 constexpr size_t kNoAllocBytes = size_t(64) << 20;
-constexpr int kMaxDevices = 64;
-constexpr int kAttemptsNoAlloc = 4;
 
 // The work space.  In host code this name is only a stand-in for the symbol:
 // the device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// The scratch array's device address on the current device (looked up once).
+// The scratch array's device address on the current device, looked up anew
+// on every call (a lookup allocates nothing).
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return cudaSuccess;
+  *out = nullptr;
+  return cudaGetSymbolAddress(out, g_noalloc_scratch);
 }
 
 // Carve the work space for `chunk` matrices of side S out of the array.
@@ -186,7 +173,7 @@ extern "C" shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, f
   for (int c0 = 0; c0 < batch && e == cudaSuccess; c0 += chunk) {
     int nm = batch - c0 < chunk ? batch - c0 : chunk;
     fill_mats_kernel<<<(nm + 127) / 128, 128, 0, st>>>(mats, nm, c0, n, p);
-    for (int attempt = 0; attempt < kAttemptsNoAlloc && nm > 0 && e == cudaSuccess; ++attempt) {
+    for (int attempt = 0; attempt < kNewtonAttempts && nm > 0 && e == cudaSuccess; ++attempt) {
       launch_newton_reset(nm, w, st);
       launch_newton_bound(A, (int64_t)n * n, n, 0, mats, nm, S, eps, attempt, w, st);
       launch_newton_init(A, (int64_t)n * n, n, 0, mats, nm, S, w, st);
@@ -206,7 +193,7 @@ extern "C" shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, f
       compact_diverged_kernel<<<1, 32, 0, st>>>(mats, nm, w, retry, nretry);
       int nr = 0;
       if ((e = read_int(nretry, &nr, st)) != cudaSuccess) break;
-      const int final_pass = (attempt == kAttemptsNoAlloc - 1) || nr == 0;
+      const int final_pass = (attempt == kNewtonAttempts - 1) || nr == 0;
       launch_newton_finalize(X, (int64_t)n * n, n, mats, nm, S, w, nullptr, iters, final_pass, st);
       count_failed_kernel<<<1, 32, 0, st>>>(nm, w, final_pass, failed);
       if (final_pass) break;

@@ -7,14 +7,19 @@ data; each step then
 
   1. reduce-scatters the gradients: one collective over a buffer laid out by
      owner leaves on each rank the sum, over ranks, of the gradients of the
-     parameters it owns, scaled by 1/world (the data-parallel mean);
+     parameters it owns, scaled by 1/world (the data-parallel mean).  The
+     buffer is float32 whatever the gradient dtype: bf16 gradients are
+     upcast (exactly) into it, summed and scaled in float32, and the owner
+     runs on the float32 mean, so no rank's contribution is rounded to bf16;
   2. runs update_stats, compute_roots (when due) and apply for its own
      parameters through its own library context -- a parameter's blocks and
      its layer-wise graft norms never leave its owner;
   3. all-gathers the updated weights, so every rank holds the whole model.
 
 Collective bytes per rank and step: the gradient buffer (world x the largest
-owner share, in the gradient dtype) and the weight buffer (the same, float32).
+owner share, float32) and the weight buffer (the same, float32).  With one
+process the gradients pass through in their own dtype (the mean of one
+gradient is itself).
 Ownership comes from shampoo_plan_shards, which every rank evaluates to the
 same plan.  With one process (no process group) the collectives are skipped.
 """
@@ -54,18 +59,20 @@ class ShardedShampoo:
             size[o] += -(-self.numel[i] // _ALIGN) * _ALIGN
         self.pad = max(max(size), _ALIGN)
         self.mine = [i for i, o in enumerate(self.owner) if o == self.rank]
+        # the dtype the owners receive: the float32 mean across ranks, or the
+        # gradient itself in one process
+        local_dtype = grad_dtype if self.world == 1 else "f32"
         if make_local is None:
             from .optimizer import Shampoo
 
             def make_local(sh):
-                return Shampoo(sh, block_size, beta2, eps, p, graft, momentum, grad_dtype, stream)
+                return Shampoo(sh, block_size, beta2, eps, p, graft, momentum, local_dtype, stream)
         self.local = make_local([self.shapes[i] for i in self.mine]) if self.mine else None
-        self.gdtype = torch.bfloat16 if grad_dtype == "bf16" else torch.float32
+        self.gdtype = torch.bfloat16 if local_dtype == "bf16" else torch.float32
         self._bufs = None
 
     def collective_bytes_per_step(self):
-        g = 2 if self.gdtype.itemsize == 2 else 4
-        return self.world * self.pad * (g + 4)
+        return 0 if self.world == 1 else self.world * self.pad * (4 + 4)
 
     def _buffers(self, device):
         import torch

@@ -605,3 +605,40 @@ def test_stalled_pipeline_wait_is_reported_and_the_context_survives():
     X, iters = batched_inverse_root(A, 2, 1e-6)
     assert int(iters[0]) >= 0
     assert torch.allclose(X[0], torch.eye(64, device="cuda") * (4.0 + 1e-6) ** -0.5)
+
+
+@pytest.mark.parametrize("gdtype", ["f32", "bf16"])
+def test_statistics_gemm_timeout_is_reported_by_the_step_calls(gdtype):
+    """The statistics GEMM of one update_stats is made to stall (its MMA
+    issuer waits once on a barrier phase nothing completes): the launch runs
+    out its bounded wait, aborts and sets the error word.  compute_roots, the
+    next synchronising call, returns SHAMPOO_ECUDA, and so do the later calls
+    on that context; a fresh context on the same device then matches the
+    oracle (the abort faulted nothing).  bf16 gradients also exercise the
+    statistics tile staged through shared memory by TMA."""
+    import time
+    from shampoo_second_order_b200 import Shampoo, _lib
+    shapes = [(300, 200), (64,)]
+    opt = Shampoo(shapes, 128, 0.99, 1e-6, 4, 1, 0.0, gdtype)
+    g = [to_dev(x, gdtype) for x in wl.make_grads(shapes, 31, 0, 1e-2, gdtype)]
+    W = [torch.from_numpy(w).cuda() for w in wl.make_params(shapes, 31)]
+    opt.update_stats(g)
+    opt.compute_roots()
+    opt.apply(W, g, 0.1)
+    _lib.shampoo_selftest_stall_next_stats(opt.ctx)
+    t0 = time.time()
+    opt.update_stats(g)                      # asynchronous: returns before the kernel ends
+    with pytest.raises(_lib.ShampooError) as e:
+        opt.compute_roots()
+    assert e.value.status == _lib.ECUDA and "timed out" in str(e.value)
+    assert time.time() - t0 < 60
+    with pytest.raises(_lib.ShampooError) as e:
+        opt.root_status()
+    assert e.value.status == _lib.ECUDA
+    for call in (lambda: opt.update_stats(g), lambda: opt.apply(W, g, 0.1)):
+        with pytest.raises(_lib.ShampooError) as e:
+            call()
+        assert e.value.status == _lib.ECUDA
+    opt.close()
+    w = run_pair(shapes, 128, 0.99, 1e-6, 1, 0.0, 0.1, gdtype, steps=3, interval=2, seed=31, gstd=1e-2)
+    assert_worst(w)

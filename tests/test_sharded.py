@@ -90,11 +90,11 @@ SHAPES = [(70, 40), (33,), (40, 90), (8, 8), (130,), (64, 64), (1, 50)]
 CFG = dict(b=32, beta2=0.95, eps=1e-2, graft=1, mu=0.5, lr=0.05, steps=5, interval=2)
 
 
-def _rank_grads(rank, t):
-    return wl.make_grads(SHAPES, 100 + rank, t, 1e-1, "f32")
+def _rank_grads(rank, t, dtype="f32"):
+    return wl.make_grads(SHAPES, 100 + rank, t, 1e-1, dtype)
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, dtype="f32"):
     import torch
     import torch.distributed as dist
     from datetime import timedelta
@@ -104,19 +104,21 @@ def _worker(rank, world, port, q):
     from shampoo_second_order_b200.sharded import ShardedShampoo
     c = CFG
     opt = ShardedShampoo(SHAPES, c["b"], c["beta2"], c["eps"], graft=c["graft"], momentum=c["mu"],
-                         root_interval=c["interval"],
+                         grad_dtype=dtype, root_interval=c["interval"],
                          make_local=lambda sh: OracleLocal(sh, c["b"], c["beta2"], c["eps"], c["graft"], c["mu"]))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     ref = ShampooOracle(SHAPES, c["b"], c["beta2"], c["eps"], 4, c["graft"], c["mu"])
     W0 = wl.make_params(SHAPES, 5)
     W = [torch.from_numpy(w.astype(np.float32)) for w in W0]
     Wr = [w.astype(np.float32).astype(np.float64) for w in W0]
     worst = 0.0
     for t in range(c["steps"]):
-        mine = _rank_grads(rank, t)
-        mean = [sum(_rank_grads(r, t)[i].astype(np.float64) for r in range(world)) / world
+        mine = _rank_grads(rank, t, dtype)
+        # the exact mean of the ranks' gradients (bf16 values held exactly)
+        mean = [sum(_rank_grads(r, t, dtype)[i].astype(np.float64) for r in range(world)) / world
                 for i in range(len(SHAPES))]
         roots = t % c["interval"] == 0
-        opt.step(W, [torch.from_numpy(g) for g in mine], c["lr"], roots)
+        opt.step(W, [torch.from_numpy(g).to(tdt) for g in mine], c["lr"], roots)
         Wr = ref.step(Wr, mean, c["lr"], roots)
         for w, r_ in zip(W, Wr):
             d = np.abs(w.double().numpy() - r_).max() / max(np.abs(r_).max(), 1e-30)
@@ -131,12 +133,14 @@ def _worker(rank, world, port, q):
     q.put((rank, worst, same, opt.mine, opt.collective_bytes_per_step()))
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sharded_step_matches_one_oracle_on_mean_gradients(world):
+@pytest.mark.parametrize("world,dtype", [(2, "f32"), (3, "f32"), (2, "bf16"), (3, "bf16")])
+def test_sharded_step_matches_one_oracle_on_mean_gradients(world, dtype):
+    """bf16 gradients are summed in float32: a bf16 reduction would round
+    each partial sum to 8 bits and miss the 1e-6 bar by orders of magnitude."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, dtype)) for r in range(world)]
     for p in procs:
         p.start()
     out = [q.get(timeout=300) for _ in procs]
