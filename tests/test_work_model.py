@@ -77,19 +77,49 @@ def test_job_throughput_is_total_work_over_the_slowest_rank():
     assert abs(bench.job_tflops(1e12, 4, 2.0) - 2000.0) < 1e-9
 
 
-def test_committed_dram_traffic_is_reported_only_for_its_workload():
+def test_committed_dram_traffic_is_reported_only_for_its_workload(monkeypatch):
     """The ncu traffic per launch was captured on one workload; the roofline
     block carries it there and null everywhere else."""
+    monkeypatch.setitem(bench.TRAFFIC_PER_LAUNCH, ("transformer_layer_b512", "newton_step_a"), 123)
     peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}
     for name, key, expect in [("transformer_layer_b512", "transformer_layer_b512", True),
                               ("transformer_big_b1024", "transformer_big_b1024", False),
                               ("transformer_layer_b512", None, False)]:
         c = wl.CONFIGS[name]
         n = len(bench.matrix_sizes(c))
-        prof = {"newton_step_a": (9, 5.0), "stats_tc": (20, 1.0)}
-        top, roof = bench.roofline(c, prof, [7] * n, 20, 1, peaks, 35.0, 6, key)
+        prof = {"newton_step_a": (9, 50.0), "stats_tc": (20, 1.0)}
+        top, roof, every = bench.roofline(c, prof, [7] * n, 20, 1, peaks, 35.0, 6, key)
         assert top == "newton_step_a" and roof["bound"] == "tensor"
         assert (roof["traffic"] is not None) == expect
+        assert set(every) == {"newton_step_a", "stats_tc"}
         # achieved = the launches' credited products over their event time
         a = bench.newton_flops(c, [7] * n, per_kernel=True)[0]
-        assert abs(roof["achieved"] - a / 5e-3 / 1e12) < 1e-3 * roof["achieved"]
+        assert abs(roof["achieved"] - a / 50e-3 / 1e12) < 1e-3 * roof["achieved"]
+
+
+def test_the_dominant_kernel_is_taken_on_the_amortised_step():
+    """Root kernels count once per root interval: 5 ms of Newton in one root
+    step of a 100-step interval weighs 0.05 ms per step, less than a 0.5 ms
+    statistics GEMM that runs every step."""
+    c = wl.CONFIGS["transformer_big_b1024"]
+    n = len(bench.matrix_sizes(c))
+    prof = {"newton_step_a": (9, 5.0), "stats_tc": (20, 10.0)}
+    am = bench.amortised_ms(prof, 20, 1, c["root_interval"])
+    assert abs(am["newton_step_a"] - 0.05) < 1e-12 and abs(am["stats_tc"] - 0.5) < 1e-12
+    top, roof, _ = bench.roofline(c, prof, [5] * n, 20, 1, {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}, 35.0)
+    assert top == "stats_tc"
+
+
+def test_both_arms_credit_the_same_step_work():
+    """The credited work of an amortised step: statistics + apply + the
+    credited Newton steps of every iterated statistic over the interval (a
+    dropped one-sided factor is not iterated)."""
+    c = wl.CONFIGS["transformer_big_b1024"]
+    k = bench.NEWTON_STEPS_CREDIT["transformer_big_b1024"]
+    f = 1024 * 1024 * 1025
+    # 544 statistics of side 1024, p = 4: per step X T (less the first), T T, T2 T2, T4 M
+    roots = 544 * (4 * k - 1) * f
+    assert bench.credited_step_flops(c, "transformer_big_b1024") == (
+        bench.stats_flops(c) + bench.apply_flops(c) + roots / 100)
+    one = dict(wl.CONFIGS["single_64x32"], right_only=[0])
+    assert bench.credit_iters(one, 6) == [0, 6]
