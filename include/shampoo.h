@@ -404,6 +404,22 @@ shampoo_status shampoo_plan_shards(int nparams, const int64_t* shapes,
                                    double* rank_cost);
 
 /*
+ * shampoo_set_gemm_tiles -- the tiling of the statistics and apply GEMMs.
+ *  pair = 1 (the default): where the block side is a multiple of 256, the two
+ *    apply GEMMs run 256 x 256 output tiles on pairs of CTAs (tcgen05
+ *    cta_group::2: each CTA of a pair loads half of each operand tile, one
+ *    MMA reads both), which halves the operand bytes each SM reads per
+ *    output.
+ *  pair = 0: 128 x 128 tiles on single CTAs.
+ * The statistics GEMM always runs single-CTA 128 x 128 tiles (its two-level
+ * accumulation keeps 128 running sums per thread).  Both tilings compute the
+ * same products in the same precision scheme (results agree to rounding
+ * order).  Takes effect from the next call.  SHAMPOO_EINVAL for any other
+ * value.
+ */
+shampoo_status shampoo_set_gemm_tiles(shampoo_ctx* ctx, int pair);
+
+/*
  * shampoo_selftest_stalled_wait -- failure-path check: launches one warp
  * that waits, through the same bounded mbarrier wait every tensor-core
  * pipeline of the library uses, on a barrier phase that nothing completes.
@@ -431,6 +447,18 @@ shampoo_status shampoo_selftest_stalled_wait(void* stream);
  * no fault, no hang.  SHAMPOO_EINVAL if ctx is NULL.
  */
 shampoo_status shampoo_selftest_stall_next_stats(shampoo_ctx* ctx);
+
+/*
+ * shampoo_selftest_stall_next_apply -- the same failure-path check for the
+ * apply GEMMs: the next shampoo_apply launches its first GEMM (Y = G R^{-1/p},
+ * on CTA pairs where the block side is a multiple of 256) with the MMA issuer
+ * first waiting on a barrier phase that nothing completes; the launch aborts
+ * as above (both CTAs of a pair together), the weights of that step are not
+ * valid, and the next synchronising call -- or the next step call, once the
+ * error word has been copied back -- returns SHAMPOO_ECUDA.  SHAMPOO_EINVAL if
+ * ctx is NULL.
+ */
+shampoo_status shampoo_selftest_stall_next_apply(shampoo_ctx* ctx);
 
 /* Library version, "MAJOR.MINOR.PATCH". */
 const char* shampoo_version(void);

@@ -54,6 +54,8 @@ SIGNATURES = {
                                       C.c_int, C.POINTER(C.c_int32), C.POINTER(C.c_double)]),
     "shampoo_selftest_stalled_wait": (C.c_int, [_P]),
     "shampoo_selftest_stall_next_stats": (C.c_int, [_P]),
+    "shampoo_set_gemm_tiles": (C.c_int, [_P, C.c_int]),
+    "shampoo_selftest_stall_next_apply": (C.c_int, [_P]),
     "shampoo_version": (C.c_char_p, []),
 }
 
@@ -251,8 +253,16 @@ def shampoo_plan_shards(shapes, block_size, root_interval, nranks):
     return list(owner), list(cost)
 
 
+def shampoo_set_gemm_tiles(ctx, pair):
+    return _check(lib().shampoo_set_gemm_tiles(ctx, int(pair)), ctx)
+
+
 def shampoo_selftest_stall_next_stats(ctx):
     return _check(lib().shampoo_selftest_stall_next_stats(ctx), ctx)
+
+
+def shampoo_selftest_stall_next_apply(ctx):
+    return _check(lib().shampoo_selftest_stall_next_apply(ctx), ctx)
 
 
 def shampoo_version():

@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libshampoo_b200.so")
-SOURCES = ["api.cu", "k_stats.cu", "k_roots.cu", "k_apply.cu", "k_tc.cu", "k_ozaki.cu", "noalloc.cu", "plan.cu"]
+SOURCES = ["api.cu", "k_stats.cu", "k_roots.cu", "k_apply.cu", "k_tc.cu", "k_tc2.cu", "k_ozaki.cu", "noalloc.cu", "plan.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

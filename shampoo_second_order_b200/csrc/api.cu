@@ -179,6 +179,8 @@ struct shampoo_ctx {
   OzakiMaps oz{};                          // over nw.q, once allocated
   int* h_count = nullptr;   // pinned [3]: Newton counts [0..1], a copy of the error word [2]
   int stall_next_stats = 0;  // failure-path test: the next statistics GEMM stalls and aborts
+  int stall_next_apply = 0;  // failure-path test: the next apply's first GEMM stalls and aborts
+  int pair_tiles = 1;        // 256 x 256 CTA-pair tiles for the apply GEMMs where the block side allows
   cudaEvent_t ev[2] = {nullptr, nullptr};
   std::vector<void*> allocs;
 
@@ -917,8 +919,8 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
   if (nblk) {
     cudaError_t e = cudaSuccess;
     run(pr, "stats_tc", s, [&] {
-      e = launch_stats_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S,
-                          ctx->planes_g, ctx->beta2, ctx->stats, ctx->d_err, s, ctx->stall_next_stats);
+      e = launch_stats_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S, ctx->planes_g,
+                          ctx->beta2, ctx->stats, ctx->d_err, s, ctx->stall_next_stats);
     });
     ctx->stall_next_stats = 0;
     if (e != cudaSuccess) return cuda_fail(ctx, e, "stats_tc");
@@ -1059,14 +1061,20 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
     shampoo_status gs = gather(ctx, grads, false);
     if (gs != SHAMPOO_OK) return gs;
     cudaError_t e = cudaSuccess;
+    const bool pair = ctx->pair_tiles && pair_gemm_supported(ctx->S);
     run(pr, "apply_y_tc", s, [&] {
-      e = launch_apply_y_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S,
-                            ctx->planes_g, ctx->yplanes, ctx->d_err, s);
+      e = pair ? launch_apply_y_pair(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S, ctx->planes_g,
+                                     ctx->yplanes, ctx->d_err, s, ctx->stall_next_apply)
+               : launch_apply_y_tc(ctx->maps, ctx->d_blocks, ctx->flags, nblk, ctx->nmat, ctx->S,
+                                   ctx->planes_g, ctx->yplanes, ctx->d_err, s, ctx->stall_next_apply);
     });
+    ctx->stall_next_apply = 0;
     if (e != cudaSuccess) return cuda_fail(ctx, e, "apply_y_tc");
     run(pr, "apply_p_tc", s, [&] {
-      e = launch_apply_p_tc(ctx->maps, ctx->d_blocks, ctx->d_params, ctx->flags, nblk, ctx->nmat,
-                            ctx->S, ctx->P, ctx->p2, ctx->d_err, s);
+      e = pair ? launch_apply_p_pair(ctx->maps, ctx->d_blocks, ctx->d_params, ctx->flags, nblk, ctx->nmat, ctx->S,
+                                     ctx->P, ctx->p2, ctx->d_err, s)
+               : launch_apply_p_tc(ctx->maps, ctx->d_blocks, ctx->d_params, ctx->flags, nblk, ctx->nmat,
+                                   ctx->S, ctx->P, ctx->p2, ctx->d_err, s);
     });
     if (e != cudaSuccess) return cuda_fail(ctx, e, "apply_p_tc");
   }
@@ -1164,9 +1172,22 @@ shampoo_status shampoo_set_one_sided(shampoo_ctx* ctx, int param, int side) {
   return SHAMPOO_OK;
 }
 
+shampoo_status shampoo_set_gemm_tiles(shampoo_ctx* ctx, int pair) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  if (pair != 0 && pair != 1) return fail(ctx, SHAMPOO_EINVAL, "pair must be 0 or 1");
+  ctx->pair_tiles = pair;
+  return SHAMPOO_OK;
+}
+
 shampoo_status shampoo_selftest_stall_next_stats(shampoo_ctx* ctx) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   ctx->stall_next_stats = 1;
+  return SHAMPOO_OK;
+}
+
+shampoo_status shampoo_selftest_stall_next_apply(shampoo_ctx* ctx) {
+  if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
+  ctx->stall_next_apply = 1;
   return SHAMPOO_OK;
 }
 

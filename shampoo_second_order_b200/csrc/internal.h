@@ -74,10 +74,20 @@ cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const i
                             int nmat, int S, int planes_g, float beta2, float* stats, int* err,
                             cudaStream_t s, int stall = 0);
 cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
-                              int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s);
+                              int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s,
+                              int stall = 0);
 cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const ParamDesc* params,
                               const int* flags, int nblk, int nmat, int S, float* P, double* p2,
                               int* err, cudaStream_t s);
+
+// ---------------- the apply GEMMs on CTA pairs, 256 x 256 tiles (k_tc2.cu) ----------------
+bool pair_gemm_supported(int S);   // S a multiple of 256
+// stall != 0 (failure-path test only): as for launch_stats_tc
+cudaError_t launch_apply_y_pair(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk, int nmat,
+                                int S, int planes_g, uint16_t* y, int* err, cudaStream_t s, int stall = 0);
+cudaError_t launch_apply_p_pair(const TcMaps& maps, const BlockDesc* blocks, const ParamDesc* params,
+                                const int* flags, int nblk, int nmat, int S, float* P, double* p2, int* err,
+                                cudaStream_t s);
 
 // ---------------- stats (k_stats.cu) ----------------
 void launch_check_finite(const ChunkDesc* chunks, int nchunks, const void* const* gptr,

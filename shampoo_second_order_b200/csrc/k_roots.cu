@@ -525,7 +525,9 @@ __global__ void __launch_bounds__(256) newton_t0_kernel(const NewtonMat* __restr
 //   job 0: X_next = X T      job 1: T2 = T T            (launch A)
 //   T4 = T2 T2 (p = 4 only)                              (launch B)
 //   M_next = T^p M, residual, T <- ((p+1) I - M_next)/p  (launch C)
-// grid: x = upper-triangular tile, y = matrix, z = job.
+// grid: x = upper-triangular tile (x 2 jobs in launch A), y = matrix.  The
+// two jobs of a tile are neighbours in launch order, so they run side by
+// side and read the tile's column panel of T from L2 once between them.
 // ---------------------------------------------------------------------------
 template <int TT>
 __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
@@ -535,13 +537,14 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
   if ((int)blockIdx.y >= w.count[2]) return;   // the check listed fewer
   const int m = w.live[blockIdx.y];
   const int st = w.state[m];
-  if (st != kRunning && !(st == kFinal && blockIdx.z == 0)) return;
+  const int job = blockIdx.x & 1;
+  if (st != kRunning && !(st == kFinal && job == 0)) return;
   const int T = S / TT;
   int ti, tj;
-  tri_tile(blockIdx.x, T, ti, tj);
+  tri_tile(blockIdx.x >> 1, T, ti, tj);
   const size_t base = (size_t)m * S * S;
   const double* Tm = w.T + base;
-  if (blockIdx.z == 0 && it == 0) {
+  if (job == 0 && it == 0) {
     // X0 = c^{-1} I, so X1 = s_0^{1/p} c^{-1} T0 needs no product: the tile
     // and its mirror (T0 is stored whole) are copied, scaled
     const double sk = sched_at(w, m, 0);
@@ -555,11 +558,11 @@ __global__ void __launch_bounds__(kNewtonThreads, 4) newton_step_a_kernel(
     }
     return;
   }
-  const double* A = blockIdx.z == 0 ? w.X[it & 1] + base : Tm;
-  double* C = blockIdx.z == 0 ? w.X[(it + 1) & 1] + base : w.T2 + base;
+  const double* A = job == 0 ? w.X[it & 1] + base : Tm;
+  double* C = job == 0 ? w.X[(it + 1) & 1] + base : w.T2 + base;
   double acc[FM][FM][2] = {};
   dmma_tile<TT>(A, Tm, S, ti * TT, tj * TT, acc, sm);
-  if (blockIdx.z == 0) {   // X_next = s_k^{1/p} X T
+  if (job == 0) {   // X_next = s_k^{1/p} X T
     const double sk = sched_at(w, m, it);
     if (sk != 1.0) {
       const double mu = pow(sk, 1.0 / mats[m].p);
@@ -807,9 +810,9 @@ static int num_tri(int S, int tile) {
 void launch_newton_step_a(const NewtonMat* mats, int rows, int S, int it, int tile, NewtonWork w, cudaStream_t s) {
   if (rows < 1) return;
   if (tile == 32)
-    newton_step_a_kernel<32><<<dim3(num_tri(S, 32), rows, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+    newton_step_a_kernel<32><<<dim3(2 * num_tri(S, 32), rows), kNewtonThreads, 0, s>>>(mats, S, it, w);
   else
-    newton_step_a_kernel<64><<<dim3(num_tri(S, 64), rows, 2), kNewtonThreads, 0, s>>>(mats, S, it, w);
+    newton_step_a_kernel<64><<<dim3(2 * num_tri(S, 64), rows), kNewtonThreads, 0, s>>>(mats, S, it, w);
 }
 
 void launch_newton_step_b(const NewtonMat* mats, int rows, int S, int tile, NewtonWork w, cudaStream_t s) {

@@ -33,6 +33,14 @@ namespace {
 constexpr int kTM = 128;          // output tile side (M = N = 128)
 constexpr int kBKe = 64;          // K elements per stage (one 128-byte row)
 constexpr int kBoxBytes = kTM * kBKe * 2;   // 16 KB: one operand plane per stage
+#ifndef SHAMPOO_STATS_CHUNK_STAGES
+#define SHAMPOO_STATS_CHUNK_STAGES 1
+#endif
+constexpr int kChunkStages = SHAMPOO_STATS_CHUNK_STAGES;   // statistics: K stages per accumulation chunk
+#ifndef SHAMPOO_STATS_CORR_FIRST
+#define SHAMPOO_STATS_CORR_FIRST 1
+#endif
+constexpr bool kCorrFirst = SHAMPOO_STATS_CORR_FIRST != 0;
 
 enum : int { kStats = 0, kApplyY = 1, kApplyP = 2 };
 
@@ -140,7 +148,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   } else {
     npass = 3; pas = (1u << 4); pbs = (1u << 2);          // h h, h l, l h
   }
-  const int stage_bytes = (nA + nB) * kBoxBytes;
+  // at S <= 128 every statistics tile is diagonal (its B operand is the A
+  // panel), so a stage holds the A planes only and twice as many fit
+  const int stage_bytes = (MODE == kStats && S <= kTM ? nA : nA + nB) * kBoxBytes;
   // bf16 statistics: the old statistics tile comes in by TMA during the main
   // loop, is updated in shared memory and goes back out by TMA
   const bool cstage = (MODE == kStats) && g1;
@@ -247,53 +257,62 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       *abort_flag = 1;
       atomicExch(args.err, tc::kErrTimeout);
     }
-    int g = 0, i = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+    int g = 0, i = 0;   // i counts accumulation items: (tile, K chunk)
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok && !*abort_flag; t += gridDim.x) {
       const TileInfo x = decode_tile<MODE>(t, args);
       if (x.skip) continue;
       const int a_mn = (MODE == kStats) ? x.isR : 0;
       const int b_mn = (MODE == kStats) ? x.isR : (MODE == kApplyP);
       const bool diag = (MODE == kStats) && x.i0 == x.j0;   // B operand = the A panel
       const uint32_t idesc = tc::idesc_bf16(kTM, kTM, a_mn, b_mn);
-      const int acc = i & 1;
-      if (i >= 2 && !tc::mbar_wait(&tempty[acc], ((i >> 1) - 1) & 1)) {
-        *abort_flag = 1;
-        atomicExch(args.err, tc::kErrTimeout);
-        break;
-      }
-      tc::fence_after_sync();
-      const uint32_t dt = tmem + acc * kTM;
       const int nk = (x.K + kBKe - 1) / kBKe;
-      bool ok = true;
-      for (int kt = 0; kt < nk; ++kt, ++g) {
-        const int s = g % ST;
-        if (!tc::mbar_wait(&full[s], (g / ST) & 1)) {
+      // stages per accumulation chunk (bf16 gradients: one product per stage, twice as deep)
+      const int cs = (MODE == kStats) ? (g1 ? 2 : 1) * kChunkStages : nk;
+      for (int c0 = 0; c0 < nk && ok; c0 += cs, ++i) {
+        const int acc = i & 1;
+        if (i >= 2 && !tc::mbar_wait(&tempty[acc], ((i >> 1) - 1) & 1)) {
           *abort_flag = 1;
           atomicExch(args.err, tc::kErrTimeout);
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t st = tc::smem_u32(smem + s * stage_bytes);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          for (int q = 0; q < npass; ++q) {
-            const int pa = (pas >> (2 * q)) & 3;
-            const int pb = (pbs >> (2 * q)) & 3;
-            const uint32_t sa = st + pa * kBoxBytes;
-            const uint32_t sb = st + (diag ? pb : nA + pb) * kBoxBytes;
-            const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
-                                     : tc::smem_desc(sa + kk * 32, 16, 1024);
-            const uint64_t db = b_mn ? tc::smem_desc(sb + kk * 2048, 8192, 1024)
-                                     : tc::smem_desc(sb + kk * 32, 16, 1024);
-            tc::mma_bf16(dt, da, db, idesc, (kt | kk | q) != 0);
+        const uint32_t dt = tmem + acc * kTM;
+        const int c1 = c0 + cs < nk ? c0 + cs : nk;
+        for (int kt = c0; kt < c1; ++kt, ++g) {
+          const int s = g % ST;
+          if (!tc::mbar_wait(&full[s], (g / ST) & 1)) {
+            *abort_flag = 1;
+            atomicExch(args.err, tc::kErrTimeout);
+            ok = false;
+            break;
           }
+          tc::fence_after_sync();
+          const uint32_t st = tc::smem_u32(smem + s * stage_bytes);
+          // statistics: a stage's small split products (hm mh hl mm lh) go
+          // into the accumulator before its large h h products, while the
+          // running sum is still small, so their truncation costs less
+          for (int qq = 0; qq < npass; ++qq) {
+            const int q = (MODE == kStats && kCorrFirst) ? (qq + 1 < npass ? qq + 1 : 0) : qq;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int pa = (pas >> (2 * q)) & 3;
+              const int pb = (pbs >> (2 * q)) & 3;
+              const uint32_t sa = st + pa * kBoxBytes;
+              const uint32_t sb = st + (diag ? pb : nA + pb) * kBoxBytes;
+              const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
+                                       : tc::smem_desc(sa + kk * 32, 16, 1024);
+              const uint64_t db = b_mn ? tc::smem_desc(sb + kk * 2048, 8192, 1024)
+                                       : tc::smem_desc(sb + kk * 32, 16, 1024);
+              tc::mma_bf16(dt, da, db, idesc, ((kt - c0) | kk | qq) != 0);
+            }
+          }
+          tc::mma_commit(&empty[s]);
         }
-        tc::mma_commit(&empty[s]);
+        if (!ok) break;
+        tc::mma_commit(&tfull[acc]);
       }
-      if (!ok) break;
-      tc::mma_commit(&tfull[acc]);
-      ++i;
     }
     // every MMA this thread issued has landed before TMEM is released
     tc::mma_commit(drain);
@@ -301,7 +320,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> registers -> global ----------------
     const int q = warp & 3;                      // TMEM lanes 32q .. 32q + 31
-    int i = 0;
+    int i = 0;         // accumulation items: (tile, K chunk)
+    int nt = 0;        // tiles finished (the phase of the statistics-tile barriers)
     int c_loads = 0;   // statistics-tile loads issued (phase of the next one)
     // bf16 statistics: lane 0 of warp 2 owns the shared statistics tile; it
     // loads the first tile's old statistics now and each next tile's right
@@ -320,25 +340,101 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       }
     };
     if (cstage && warp == 2 && lane == 0) load_c(blockIdx.x);
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
       const TileInfo x = decode_tile<MODE>(t, args);
       if (x.skip) continue;
-      const int acc = i & 1;
-      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&tfull[acc], (i >> 1) & 1) && !*abort_flag);
-      if (!ok) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          atomicExch(args.err, tc::kErrTimeout);
-        }
-        break;
-      }
-      tc::fence_after_sync();
       const int blk = x.blk, i0 = x.i0, j0 = x.j0;
       const BlockDesc bd = args.blocks[blk];
       const int r = i0 + q * 32 + lane;          // output row owned by this thread
-      const uint32_t trow = tmem + acc * kTM + ((uint32_t)(q * 32) << 16);
+      const int nk = (x.K + kBKe - 1) / kBKe;
+      const int cs = (MODE == kStats) ? (g1 ? 2 : 1) * kChunkStages : nk;
+      float sum[MODE == kStats ? 128 : 1];       // statistics: this row of the tile over the chunks
+      for (int c0 = 0; c0 < nk; c0 += cs, ++i) {
+        const int acc = i & 1;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait_sleepy(&tfull[acc], (i >> 1) & 1) && !*abort_flag);
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            atomicExch(args.err, tc::kErrTimeout);
+          }
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t trow = tmem + acc * kTM + ((uint32_t)(q * 32) << 16);
+        if (MODE == kStats) {
+          const bool first = c0 == 0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tc::tmem_ld32(trow + c * 32, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int k = MODE == kStats ? 32 * c + e : 0;
+              sum[k] = (first ? 0.f : sum[k]) + v[e];
+            }
+          }
+        } else if (MODE == kApplyY) {
+          uint16_t* yh = args.y + (size_t)blk * S * S;
+          uint16_t* yl = args.y + (size_t)(args.nblk + blk) * S * S;
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tc::tmem_ld32(trow + c * 32, v);
+            const int cb = j0 + c * 32;
+            if (r < S && cb < S) {
+              uint32_t hw[16], lw[16];
+  #pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                const uint16_t h0 = tc::bf16_bits_rn(v[2 * u]), h1 = tc::bf16_bits_rn(v[2 * u + 1]);
+                const uint16_t l0 = tc::bf16_bits_rn(v[2 * u] - tc::bf16_to_f(h0));
+                const uint16_t l1 = tc::bf16_bits_rn(v[2 * u + 1] - tc::bf16_to_f(h1));
+                hw[u] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                lw[u] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+              }
+              uint4* dh = reinterpret_cast<uint4*>(yh + (size_t)r * S + cb);
+              uint4* dl = reinterpret_cast<uint4*>(yl + (size_t)r * S + cb);
+  #pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                dh[u] = make_uint4(hw[4 * u], hw[4 * u + 1], hw[4 * u + 2], hw[4 * u + 3]);
+                dl[u] = make_uint4(lw[4 * u], lw[4 * u + 1], lw[4 * u + 2], lw[4 * u + 3]);
+              }
+            }
+          }
+        } else {
+          double ss = 0.0;
+          float* Pp = args.P + args.params[bd.param].offset;
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tc::tmem_ld32(trow + c * 32, v);
+            const int cb = j0 + c * 32;
+            if (r < bd.m) {
+              float* dst = Pp + (bd.r0 + r) * bd.ld + bd.c0 + cb;
+              if (cb + 32 <= bd.n && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+  #pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+  #pragma unroll
+                for (int e = 0; e < 32; ++e) ss += (double)v[e] * v[e];
+              } else {
+  #pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  if (cb + e < bd.n) {
+                    dst[e] = v[e];
+                    ss += (double)v[e] * v[e];
+                  }
+                }
+              }
+            }
+          }
+          ss = warp_sum(ss);
+          if (lane == 0 && ss != 0.0) atomicAdd(&args.p2[bd.param], ss);
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&tempty[acc]);
+      }
+      if (!ok) break;
       if (MODE == kStats && cstage) {
-        if (!__all_sync(0xffffffffu, tc::mbar_wait(cfull, i & 1))) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(cfull, nt & 1))) {
           if (lane == 0) {
             *abort_flag = 1;
             atomicExch(args.err, tc::kErrTimeout);
@@ -347,27 +443,27 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         }
         const int rl = q * 32 + lane;            // tile-local row
         const int nbox = (S - j0 + 31) / 32 < 4 ? (S - j0 + 31) / 32 : 4;
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(trow + c * 32, v);
           if (c >= nbox) continue;
           // row rl of box c: 8 chunks of 16 B, chunk j stored at j ^ (rl & 7)
           uint8_t* row = cbuf + c * (kCTileBytes / 4) + rl * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
+            const int k = MODE == kStats ? 32 * c + 4 * j : 0;
             float4* p4 = reinterpret_cast<float4*>(row + ((j ^ (rl & 7)) << 4));
             float4 o = *p4;
-            o.x = fmaf(args.beta2, o.x, v[4 * j + 0]);
-            o.y = fmaf(args.beta2, o.y, v[4 * j + 1]);
-            o.z = fmaf(args.beta2, o.z, v[4 * j + 2]);
-            o.w = fmaf(args.beta2, o.w, v[4 * j + 3]);
+            o.x = fmaf(args.beta2, o.x, sum[k]);
+            o.y = fmaf(args.beta2, o.y, sum[k + (MODE == kStats ? 1 : 0)]);
+            o.z = fmaf(args.beta2, o.z, sum[k + (MODE == kStats ? 2 : 0)]);
+            o.w = fmaf(args.beta2, o.w, sum[k + (MODE == kStats ? 3 : 0)]);
             *p4 = o;
           }
         }
         tc::fence_proxy_async_smem();            // my writes, before the TMA store reads them
         tc::mbar_arrive(cready);
         if (warp == 2 && lane == 0) {
-          if (!tc::mbar_wait(cready, i & 1)) {
+          if (!tc::mbar_wait(cready, nt & 1)) {
             *abort_flag = 1;
             atomicExch(args.err, tc::kErrTimeout);
           } else {
@@ -380,9 +476,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         }
       } else if (MODE == kStats) {
         float* C = args.stats + (size_t)(2 * blk + x.isR) * S * S;
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(trow + c * 32, v);
           const int cb = j0 + c * 32;
           if (r < S && cb < S) {
             float4* row = reinterpret_cast<float4*>(C + (size_t)r * S + cb);
@@ -391,75 +486,20 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             for (int u = 0; u < 8; ++u) o[u] = row[u];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              o[u].x = fmaf(args.beta2, o[u].x, v[4 * u + 0]);
-              o[u].y = fmaf(args.beta2, o[u].y, v[4 * u + 1]);
-              o[u].z = fmaf(args.beta2, o[u].z, v[4 * u + 2]);
-              o[u].w = fmaf(args.beta2, o[u].w, v[4 * u + 3]);
+              const int k = MODE == kStats ? 32 * c + 4 * u : 0;
+              o[u].x = fmaf(args.beta2, o[u].x, sum[k]);
+              o[u].y = fmaf(args.beta2, o[u].y, sum[k + (MODE == kStats ? 1 : 0)]);
+              o[u].z = fmaf(args.beta2, o[u].z, sum[k + (MODE == kStats ? 2 : 0)]);
+              o[u].w = fmaf(args.beta2, o[u].w, sum[k + (MODE == kStats ? 3 : 0)]);
               row[u] = o[u];
             }
           }
         }
-      } else if (MODE == kApplyY) {
-        uint16_t* yh = args.y + (size_t)blk * S * S;
-        uint16_t* yl = args.y + (size_t)(args.nblk + blk) * S * S;
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(trow + c * 32, v);
-          const int cb = j0 + c * 32;
-          if (r < S && cb < S) {
-            uint32_t hw[16], lw[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const uint16_t h0 = tc::bf16_bits_rn(v[2 * u]), h1 = tc::bf16_bits_rn(v[2 * u + 1]);
-              const uint16_t l0 = tc::bf16_bits_rn(v[2 * u] - tc::bf16_to_f(h0));
-              const uint16_t l1 = tc::bf16_bits_rn(v[2 * u + 1] - tc::bf16_to_f(h1));
-              hw[u] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-              lw[u] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-            }
-            uint4* dh = reinterpret_cast<uint4*>(yh + (size_t)r * S + cb);
-            uint4* dl = reinterpret_cast<uint4*>(yl + (size_t)r * S + cb);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              dh[u] = make_uint4(hw[4 * u], hw[4 * u + 1], hw[4 * u + 2], hw[4 * u + 3]);
-              dl[u] = make_uint4(lw[4 * u], lw[4 * u + 1], lw[4 * u + 2], lw[4 * u + 3]);
-            }
-          }
-        }
-      } else {
-        double ss = 0.0;
-        float* Pp = args.P + args.params[bd.param].offset;
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(trow + c * 32, v);
-          const int cb = j0 + c * 32;
-          if (r < bd.m) {
-            float* dst = Pp + (bd.r0 + r) * bd.ld + bd.c0 + cb;
-            if (cb + 32 <= bd.n && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-#pragma unroll
-              for (int u = 0; u < 8; ++u)
-                reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) ss += (double)v[e] * v[e];
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                if (cb + e < bd.n) {
-                  dst[e] = v[e];
-                  ss += (double)v[e] * v[e];
-                }
-              }
-            }
-          }
-        }
-        ss = warp_sum(ss);
-        if (lane == 0 && ss != 0.0) atomicAdd(&args.p2[bd.param], ss);
       }
-      tc::fence_before_sync();
-      tc::mbar_arrive(&tempty[acc]);
-      ++i;
+      ++nt;
     }
     // after an abort a statistics-tile load may still be in flight: let it land
-    if (cstage && warp == 2 && lane == 0 && c_loads > i) tc::mbar_wait(cfull, (c_loads - 1) & 1);
+    if (cstage && warp == 2 && lane == 0 && c_loads > nt) tc::mbar_wait(cfull, (c_loads - 1) & 1);
   }
   if (cstage && warp == 2 && lane == 0) tc::bulk_wait0();   // statistics stores complete
   __syncwarp();
@@ -647,16 +687,17 @@ cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const i
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
   a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err; a.stall = stall;
   const int T = (S + kTM - 1) / kTM;
-  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, planes_g, planes_g == 1),
+  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, S <= kTM ? 0 : planes_g, planes_g == 1),
                              maps, a, s);
 }
 
 cudaError_t launch_apply_y_tc(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk,
-                              int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s) {
+                              int nmat, int S, int planes_g, uint16_t* y, int* err, cudaStream_t s,
+                              int stall) {
   if (nblk <= 0) return cudaSuccess;
   TcArgs a{};
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
-  a.planes_g = planes_g; a.y = y; a.err = err;
+  a.planes_g = planes_g; a.y = y; a.err = err; a.stall = stall;
   const int T = (S + kTM - 1) / kTM;
   return launch_mode<kApplyY>(nblk * T * T, smem_bytes(planes_g == 1 ? 1 : 2, 2), maps, a, s);
 }

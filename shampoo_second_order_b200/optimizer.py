@@ -82,6 +82,11 @@ class Shampoo:
         emulated on the int8 tensor cores with `slices` 7-bit slices)."""
         L.shampoo_set_root_method(self.ctx, _METHODS[method], slices)
 
+    def set_gemm_tiles(self, pair=True):
+        """256 x 256 CTA-pair tiles for the GEMMs where the block side allows
+        (the default), or 128 x 128 single-CTA tiles everywhere."""
+        L.shampoo_set_gemm_tiles(self.ctx, 1 if pair else 0)
+
     def set_one_sided(self, index, side):
         """Keep only one factor ("left": L, "right": R, "both": the default)
         for every block of 2-D parameter `index`; before the first step."""
