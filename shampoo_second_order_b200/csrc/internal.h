@@ -80,8 +80,9 @@ cudaError_t launch_apply_p_tc(const TcMaps& maps, const BlockDesc* blocks, const
                               const int* flags, int nblk, int nmat, int S, float* P, double* p2,
                               int* err, cudaStream_t s);
 
-// ---------------- the apply GEMMs on CTA pairs, 256 x 256 tiles (k_tc2.cu) ----------------
+// ---------------- the GEMMs on CTA pairs (k_tc2.cu) ----------------
 bool pair_gemm_supported(int S);   // S a multiple of 256
+// the apply GEMMs on 256 x 256 pair tiles
 // stall != 0 (failure-path test only): as for launch_stats_tc
 cudaError_t launch_apply_y_pair(const TcMaps& maps, const BlockDesc* blocks, const int* flags, int nblk, int nmat,
                                 int S, int planes_g, uint16_t* y, int* err, cudaStream_t s, int stall = 0);

@@ -99,8 +99,9 @@ def run_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, interval, seed
                 worst["roots"] = max(worst["roots"], rel(X, ro[k]))
         for i, s in enumerate(shapes):
             wd = Wd[i].cpu().numpy().astype(np.float64)
+            d_gpu, d_ref = wd - prev_d[i], Wo[i] - prev_o[i]   # the step, once per parameter
             for sl in pieces(s, b):
-                worst["dW"] = max(worst["dW"], rel((wd - prev_d[i])[sl], (Wo[i] - prev_o[i])[sl]))
+                worst["dW"] = max(worst["dW"], rel(d_gpu[sl], d_ref[sl]))
                 worst["W"] = max(worst["W"], rel(wd[sl], Wo[i][sl]))
     opt.close()
     return worst
@@ -449,8 +450,9 @@ def run_subset(cfg, steps, interval, keep):
     worst = {"dW": 0.0, "W": 0.0}
     for k, i in enumerate(keep):
         wd = Wd[i].cpu().numpy().astype(np.float64)
+        d_gpu, d_ref = wd - prev_d[k], Wo[k] - prev_o[k]
         for sl in pieces(shapes[i], cfg["block_size"]):
-            worst["dW"] = max(worst["dW"], rel((wd - prev_d[k])[sl], (Wo[k] - prev_o[k])[sl]))
+            worst["dW"] = max(worst["dW"], rel(d_gpu[sl], d_ref[sl]))
             worst["W"] = max(worst["W"], rel(wd[sl], Wo[k][sl]))
     opt.close()
     return worst
@@ -545,8 +547,9 @@ def run_async_pair(shapes, b, beta2, eps, graft, mu, lr, gdtype, steps, submit, 
         torch.cuda.synchronize()
         for i, s in enumerate(shapes):
             wd = Wd[i].cpu().numpy().astype(np.float64)
+            d_gpu, d_ref = wd - prev_d[i], Wo[i] - prev_o[i]   # the step, once per parameter
             for sl in pieces(s, b):
-                worst["dW"] = max(worst["dW"], rel((wd - prev_d[i])[sl], (Wo[i] - prev_o[i])[sl]))
+                worst["dW"] = max(worst["dW"], rel(d_gpu[sl], d_ref[sl]))
                 worst["W"] = max(worst["W"], rel(wd[sl], Wo[i][sl]))
     assert pending is None
     opt.close()
