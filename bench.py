@@ -53,11 +53,6 @@ UNIT = "TFLOP/s"
 # products, both factors, the default --steps/--warmup); None for any other
 # workload, mode or kernel until measured there.
 TRAFFIC_PER_LAUNCH = {
-    # the statistics GEMM (single-CTA 128x128 tiles, two-level accumulation):
-    # 283.0 MB for the 20 blocks of Transformer-big layer 0 (ncu, one launch,
-    # `python -m shampoo_second_order_b200.run_steps`), scaled by the block
-    # count to the 272 identical 1024 x 1024 blocks of a full launch
-    ("transformer_big_b1024", "stats_tc"): 283014656 * 272 // 20,
 }
 
 
@@ -300,18 +295,18 @@ def tc_work(cfg, kernel):
     b = cfg["block_size"]
     blks, _ = blocks_of(cfg)
     f32 = cfg["grad_dtype"] == "f32"
-    planes = 3 if f32 else 1
+    planes = 2 if f32 else 1
     T = (b + 127) // 128
     tri = T * (T + 1) // 2 * 128 * 128 * 4          # bytes of one statistic's upper tiles
     if kernel == "stats_tc":
-        passes = 6 if f32 else 1
+        passes = 4 if f32 else 1
         fl = sum((0 if sd else m * (m + 1) * n) + n * (n + 1) * m
                  for (m, n), sd in zip(blks, block_sides(cfg))) * passes
         by = sum(2 * planes * m * n for m, n in blks) + len(blks) * 2 * 2 * tri
     elif kernel == "apply_y_tc":
         passes = 3 if f32 else 2
         fl = sum(2 * m * n * n for m, n in blks) * passes
-        by = sum(2 * min(planes, 2) * m * n + 2 * 2 * n * n + 2 * 2 * m * n for m, n in blks)
+        by = sum(2 * planes * m * n + 2 * 2 * n * n + 2 * 2 * m * n for m, n in blks)
     else:   # apply_p_tc
         fl = sum(2 * m * m * n for m, n in blks) * 3
         by = sum(2 * 2 * m * m + 2 * 2 * m * n + 4 * m * n for m, n in blks)
@@ -377,7 +372,7 @@ def kernel_roof(cfg, name, launches, ms, iters_sum, steps, n_root_steps, peaks, 
         work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / launches, "MEASURED_PEAKS.json hbm_gbs")
     elif name in ("dnorm", "diag_update", "check_finite", "gather"):
         per = {"dnorm": gbytes + 4, "diag_update": gbytes + 8, "check_finite": gbytes,
-               "gather": gbytes + (6 if gbytes == 4 else 2)}[name]
+               "gather": gbytes + (4 if gbytes == 4 else 2)}[name]
         by = el * per * steps
         work = ("hbm", by / 1e9 / sec, hbm, "GB/s", by / launches, "MEASURED_PEAKS.json hbm_gbs")
     if work is None:

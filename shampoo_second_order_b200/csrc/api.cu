@@ -159,7 +159,7 @@ struct shampoo_ctx {
   float* a = nullptr;
   float* mom = nullptr;
   float* P = nullptr;
-  uint16_t* gblk = nullptr;     // gathered gradient planes [planes_g*nblk][S][S] (h, m, l)
+  uint16_t* gblk = nullptr;     // gathered gradient planes [planes_g*nblk][S][S] (h, m)
   uint16_t* rplanes = nullptr;  // root planes [2*nmat][S][S]
   uint16_t* yplanes = nullptr;  // Y planes [2*nblk][S][S]
   TcMaps maps{};
@@ -736,7 +736,7 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   ctx->mu = momentum;
   ctx->graft = graft;
   ctx->bf16 = grad_dtype == SHAMPOO_BF16;
-  ctx->planes_g = ctx->bf16 ? 1 : 3;
+  ctx->planes_g = ctx->bf16 ? 1 : 2;
   const int b = block_size;
 
   for (int i = 0; i < nparams; ++i) {

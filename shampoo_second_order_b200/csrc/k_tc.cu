@@ -1,6 +1,6 @@
 // Tensor-core (tcgen05) kernels of the step:
 //   gather   K1: partition each 2-D gradient into zero-padded S x S blocks as
-//                bf16 planes (fp32 gradients: hi = bf16(g), lo = bf16(g - hi))
+//                bf16 planes (fp32 gradients: h = bf16(g), m = bf16(g - h))
 //   stats    K2: L <- beta2 L + G G^T, R <- beta2 R + G^T G (transcript
 //                segment 10, first piece), upper-triangular 128 x 128 tiles
 //   apply    K4: Y = G R^{-1/p}, then P = L^{-1/p} Y (segment 10, third piece)
@@ -8,13 +8,17 @@
 //
 // Every product runs as bf16 x bf16 -> fp32 on tcgen05 with the accumulator
 // in TMEM; fp32 operands enter as sums of bf16 terms.  bf16 gradients are
-// exact in one term.  fp32 gradients are split into three terms x = h + m + l
-// (24 significant bits, exact for normal floats) and the statistics keep the
-// six products h h, h m, m h, h l, m m, l h, dropping only terms below
-// 2^-24 |x||y|: a statistic of an ill-conditioned block amplifies its own
-// error by up to its condition number in the root, so L and R need fp32
-// accuracy.  The apply products keep hi*hi + hi*lo + lo*hi of two-term
-// splits (relative error near 2^-16), well inside the step tolerance.
+// exact in one term.  fp32 gradients are split into two terms x = h + m
+// (h = bf16(x), m = bf16(x - h): x to 16 significant bits, rounded to
+// nearest) and the statistics keep all four products h h, h m, m h, m m, so
+// they are (h + m)(h + m)^T exactly up to accumulation.  What is left out,
+// h r^T + r h^T with r = x - h - m, is 2^-16 of the statistic and has no
+// sign bias (r is a round-to-nearest remainder); a positive semi-definite
+// term left out (m m^T in the three-product scheme h h + h m + m h) would
+// bias the small eigenvalues down, and an ill-conditioned block's root
+// amplifies that bias by its condition number.  The apply products keep
+// h*h + h*l + l*h of two-term splits (relative error near 2^-16), well inside
+// the step tolerance.
 //
 // The GEMM kernel is persistent and warp-specialised: one CTA per SM walks
 // the 128 x 128 output tiles round-robin with 192 threads.  Lane 0 of warp 0
@@ -49,7 +53,7 @@ struct TcArgs {
   const ParamDesc* params;
   const int* flags;
   int nblk, nmat, S;
-  int planes_g;      // 1: bf16 gradients, 3: fp32 gradients (h, m, l)
+  int planes_g;      // 1: bf16 gradients, 2: fp32 gradients (h, m)
   float beta2;
   float* stats;      // fp32 [nmat][S][S], upper 128-tiles kept
   uint16_t* y;       // bf16 planes [2][nblk][S][S], row-major Y
@@ -140,9 +144,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   if (MODE == kStats && g1) {
     npass = 1; pas = 0; pbs = 0;                          // g g
   } else if (MODE == kStats) {
-    npass = 6;                                            // hh hm mh hl mm lh
-    pas = (0u) | (0u << 2) | (1u << 4) | (0u << 6) | (1u << 8) | (2u << 10);
-    pbs = (0u) | (1u << 2) | (0u << 4) | (2u << 6) | (1u << 8) | (0u << 10);
+    npass = 4;                                            // hh hm mh mm
+    pas = (0u) | (0u << 2) | (1u << 4) | (1u << 6);
+    pbs = (0u) | (1u << 2) | (0u << 4) | (1u << 6);
   } else if (MODE == kApplyY && g1) {
     npass = 2; pas = 0; pbs = (1u << 2);                  // g R_h, g R_l
   } else {
@@ -290,9 +294,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
           }
           tc::fence_after_sync();
           const uint32_t st = tc::smem_u32(smem + s * stage_bytes);
-          // statistics: a stage's small split products (hm mh hl mm lh) go
-          // into the accumulator before its large h h products, while the
-          // running sum is still small, so their truncation costs less
+          // statistics: a stage's small split products (hm mh mm) go into
+          // the accumulator before its large h h products, while the running
+          // sum is still small, so their truncation costs less
           for (int qq = 0; qq < npass; ++qq) {
             const int q = (MODE == kStats && kCorrFirst) ? (qq + 1 < npass ? qq + 1 : 0) : qq;
 #pragma unroll
@@ -519,7 +523,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict
   const int64_t e0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (e0 >= (int64_t)S * S) return;
   const int i = (int)(e0 / S), j = (int)(e0 % S);
-  uint32_t hw[4] = {0, 0, 0, 0}, mw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
+  uint32_t hw[4] = {0, 0, 0, 0}, mw[4] = {0, 0, 0, 0};
   const void* g = gptr[bd.param];
   const int64_t base = (bd.r0 + i) * bd.ld + bd.c0;
   int bad = 0;
@@ -556,12 +560,9 @@ __global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict
         for (int q = 0; q < 8; ++q) {
           bad |= !isfinite(x[q]);
           const uint16_t h = tc::bf16_bits_rn(x[q]);
-          const float r1 = x[q] - tc::bf16_to_f(h);        // exact
-          const uint16_t m = tc::bf16_bits_rn(r1);
-          const uint16_t l = tc::bf16_bits_rn(r1 - tc::bf16_to_f(m));
+          const uint16_t m = tc::bf16_bits_rn(x[q] - tc::bf16_to_f(h));   // the difference is exact
           hw[q >> 1] |= (uint32_t)h << (16 * (q & 1));
           mw[q >> 1] |= (uint32_t)m << (16 * (q & 1));
-          lw[q >> 1] |= (uint32_t)l << (16 * (q & 1));
         }
       }
     } else {
@@ -569,7 +570,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict
       for (int q = 0; q < 8; ++q) {
         const int jj = j + q;
         if (jj < bd.n) {
-          uint16_t h, m = 0, l = 0;
+          uint16_t h, m = 0;
           if (bf16) {
             h = __ldg(reinterpret_cast<const uint16_t*>(g) + base + jj);
             bad |= (h & 0x7F80) == 0x7F80;
@@ -577,13 +578,10 @@ __global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict
             const float x = __ldg(reinterpret_cast<const float*>(g) + base + jj);
             bad |= !isfinite(x);
             h = tc::bf16_bits_rn(x);
-            const float r1 = x - tc::bf16_to_f(h);        // exact
-            m = tc::bf16_bits_rn(r1);
-            l = tc::bf16_bits_rn(r1 - tc::bf16_to_f(m));  // exact remainder, rounded
+            m = tc::bf16_bits_rn(x - tc::bf16_to_f(h));   // the difference is exact
           }
           hw[q >> 1] |= (uint32_t)h << (16 * (q & 1));
           mw[q >> 1] |= (uint32_t)m << (16 * (q & 1));
-          lw[q >> 1] |= (uint32_t)l << (16 * (q & 1));
         }
       }
     }
@@ -593,8 +591,6 @@ __global__ void __launch_bounds__(256) gather_kernel(const BlockDesc* __restrict
   *reinterpret_cast<uint4*>(out + blockIdx.y * slot + e0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
   if (!bf16) {
     *reinterpret_cast<uint4*>(out + (nblk + blockIdx.y) * slot + e0) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
-    *reinterpret_cast<uint4*>(out + (2 * (size_t)nblk + blockIdx.y) * slot + e0) =
-        make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
 }
 
