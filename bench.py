@@ -53,12 +53,6 @@ UNIT = "TFLOP/s"
 # products, both factors, the default --steps/--warmup); None for any other
 # workload, mode or kernel until measured there.
 TRAFFIC_PER_LAUNCH = {
-    # the statistics GEMM (single-CTA 128x128 tiles, 2-term split with four
-    # products, two-level accumulation): 231.4 MB for the 20 blocks of
-    # Transformer-big layer 0 (ncu, one launch, `python -m
-    # shampoo_second_order_b200.run_steps`), scaled by the block count to the
-    # 272 identical 1024 x 1024 blocks of a full launch
-    ("transformer_big_b1024", "stats_tc"): 231415296 * 272 // 20,
 }
 
 
@@ -207,7 +201,9 @@ def measured_peaks():
     if os.path.exists(p):
         with open(p) as f:
             return json.load(f), "measured"
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+    # no measured file: an earlier copy/cuBLAS measurement on B200s of this kind
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "fallback": True}, "fallback"
 
 
 class ClockSampler:
@@ -384,6 +380,8 @@ def kernel_roof(cfg, name, launches, ms, iters_sum, steps, n_root_steps, peaks, 
     if work is None:
         return None
     bound, ach, peak, unit, per_launch, src = work
+    if peaks.get("fallback"):
+        src = src.replace("MEASURED_PEAKS.json", "fallback peaks:")
     tr = TRAFFIC_PER_LAUNCH.get((traffic_key, name)) if traffic_key else None
     out = {"kernel": name, "bound": bound, "achieved": round(ach, 3), "peak": round(peak, 2),
            "unit": unit, "frac": round(ach / peak, 4), "traffic": tr,

@@ -23,10 +23,11 @@
 // The GEMM kernel is persistent and warp-specialised: one CTA per SM walks
 // the 128 x 128 output tiles round-robin with 192 threads.  Lane 0 of warp 0
 // issues TMA loads into a ring of shared-memory stages, lane 0 of warp 1
-// issues the MMAs into one of two TMEM accumulators and releases stages with
-// tcgen05.commit, and warps 2-5 drain the other accumulator (warp w owns TMEM
-// lanes 32 (w % 4) ..), so the epilogue of one tile overlaps the main loop of
-// the next.
+// issues the MMAs into a rotation of TMEM accumulators (two for the apply
+// GEMMs, four K chunks for the statistics) and releases stages with
+// tcgen05.commit, and warps 2-5 drain the finished accumulators (warp w owns
+// TMEM lanes 32 (w % 4) ..), so the epilogue of one tile overlaps the main
+// loop of the next.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -45,6 +46,10 @@ constexpr int kChunkStages = SHAMPOO_STATS_CHUNK_STAGES;   // statistics: K stag
 #define SHAMPOO_STATS_CORR_FIRST 1
 #endif
 constexpr bool kCorrFirst = SHAMPOO_STATS_CORR_FIRST != 0;
+// TMEM accumulators of the statistics GEMM (4 x 128 columns): the MMA issuer
+// may run three K chunks ahead of the epilogue, which stops draining TMEM
+// while it read-modify-writes a finished tile
+constexpr int kStatsAcc = 4;
 
 enum : int { kStats = 0, kApplyY = 1, kApplyP = 2 };
 
@@ -116,6 +121,14 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const TcArgs& a) {
 
 constexpr int kCTileBytes = 128 * 128 * 4;   // one fp32 statistics tile (4 boxes of 32 columns)
 
+// The statistics tile goes through shared memory (TMA load, update, TMA
+// store) where the ring leaves room for it: bf16 gradients (one plane per
+// operand) and S <= 128 (the stages hold the A planes only).  Elsewhere the
+// epilogue threads update it in place, one row each.
+__host__ __device__ constexpr bool stats_cstage(int planes_g, int S) {
+  return planes_g == 1 || S <= kTM;
+}
+
 // Ring stages that fit beside the 64 KB statistics tile when the update
 // stages it in shared memory (cstage), else beside nothing.
 __host__ __device__ constexpr int ring_stages(int stage_bytes, bool cstage = false) {
@@ -133,6 +146,9 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = args.S;
+  constexpr int kNAcc = (MODE == kStats) ? kStatsAcc : 2;   // TMEM accumulators
+  constexpr uint32_t kTmemCols = kNAcc * kTM <= 256 ? 256 : 512;
+  constexpr int kEpiT = 128;   // epilogue threads (warps 2-5)
 
   // operand planes loaded and the (A plane, B plane) products kept, packed
   // two bits per product
@@ -155,20 +171,20 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   // at S <= 128 every statistics tile is diagonal (its B operand is the A
   // panel), so a stage holds the A planes only and twice as many fit
   const int stage_bytes = (MODE == kStats && S <= kTM ? nA : nA + nB) * kBoxBytes;
-  // bf16 statistics: the old statistics tile comes in by TMA during the main
-  // loop, is updated in shared memory and goes back out by TMA
-  const bool cstage = (MODE == kStats) && g1;
+  // staged statistics (stats_cstage): the old statistics tile comes in by TMA
+  // during the main loop, is updated in shared memory and goes back out by TMA
+  const bool cstage = (MODE == kStats) && stats_cstage(args.planes_g, S);
   const int ST = ring_stages(stage_bytes, cstage);
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* cbuf = smem + ST * stage_bytes;     // the 64 KB statistics tile
   uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + (cstage ? kCTileBytes : 0));
   uint64_t* empty = full + ST;
-  uint64_t* tfull = empty + ST;     // [2] accumulator ready for the epilogue
-  uint64_t* tempty = tfull + 2;     // [2] accumulator drained by the epilogue
-  uint64_t* drain = tempty + 2;
+  uint64_t* tfull = empty + ST;     // [kNAcc] accumulator ready for the epilogue
+  uint64_t* tempty = tfull + 4;     // [kNAcc] accumulator drained by the epilogue
+  uint64_t* drain = tempty + 4;
   uint64_t* cfull = drain + 1;      // statistics tile loaded
-  uint64_t* cready = cfull + 1;     // all epilogue threads wrote the tile (count 128)
+  uint64_t* cready = cfull + 1;     // all epilogue threads wrote the tile
   uint64_t* never = cready + 1;     // no thread ever arrives here (the failure-path test)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -178,19 +194,19 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kNAcc; ++a) {
       tc::mbar_init(&tfull[a], 1);
-      tc::mbar_init(&tempty[a], 128);
+      tc::mbar_init(&tempty[a], kEpiT);
     }
     tc::mbar_init(drain, 1);
     tc::mbar_init(cfull, 1);
-    tc::mbar_init(cready, 128);
+    tc::mbar_init(cready, kEpiT);
     tc::mbar_init(never, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, 256);
+    tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::tmem_relinquish();
   }
   __syncthreads();
@@ -274,8 +290,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       // stages per accumulation chunk (bf16 gradients: one product per stage, twice as deep)
       const int cs = (MODE == kStats) ? (g1 ? 2 : 1) * kChunkStages : nk;
       for (int c0 = 0; c0 < nk && ok; c0 += cs, ++i) {
-        const int acc = i & 1;
-        if (i >= 2 && !tc::mbar_wait(&tempty[acc], ((i >> 1) - 1) & 1)) {
+        const int acc = i % kNAcc;
+        if (i >= kNAcc && !tc::mbar_wait(&tempty[acc], ((i / kNAcc) - 1) & 1)) {
           *abort_flag = 1;
           atomicExch(args.err, tc::kErrTimeout);
           ok = false;
@@ -327,7 +343,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
     int i = 0;         // accumulation items: (tile, K chunk)
     int nt = 0;        // tiles finished (the phase of the statistics-tile barriers)
     int c_loads = 0;   // statistics-tile loads issued (phase of the next one)
-    // bf16 statistics: lane 0 of warp 2 owns the shared statistics tile; it
+    // staged statistics: lane 0 of warp 2 owns the shared statistics tile; it
     // loads the first tile's old statistics now and each next tile's right
     // after storing the previous one, while that tile's main loop runs
     auto load_c = [&](int from) {
@@ -355,8 +371,8 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
       const int cs = (MODE == kStats) ? (g1 ? 2 : 1) * kChunkStages : nk;
       float sum[MODE == kStats ? 128 : 1];       // statistics: this row of the tile over the chunks
       for (int c0 = 0; c0 < nk; c0 += cs, ++i) {
-        const int acc = i & 1;
-        ok = __all_sync(0xffffffffu, tc::mbar_wait_sleepy(&tfull[acc], (i >> 1) & 1) && !*abort_flag);
+        const int acc = i % kNAcc;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait_sleepy(&tfull[acc], (i / kNAcc) & 1) && !*abort_flag);
         if (!ok) {
           if (lane == 0) {
             *abort_flag = 1;
@@ -480,22 +496,34 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         }
       } else if (MODE == kStats) {
         float* C = args.stats + (size_t)(2 * blk + x.isR) * S * S;
+        constexpr int NG = 2;   // column groups of 32 whose old values are loaded together
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int cb = j0 + c * 32;
-          if (r < S && cb < S) {
-            float4* row = reinterpret_cast<float4*>(C + (size_t)r * S + cb);
-            float4 o[8];
+        for (int c0 = 0; c0 < 4; c0 += NG) {
+          float4 o[8 * NG];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) o[u] = row[u];
+          for (int gq = 0; gq < NG; ++gq) {
+            const int cb = j0 + (c0 + gq) * 32;
+            if (r < S && cb < S) {
+              const float4* row = reinterpret_cast<const float4*>(C + (size_t)r * S + cb);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int k = MODE == kStats ? 32 * c + 4 * u : 0;
-              o[u].x = fmaf(args.beta2, o[u].x, sum[k]);
-              o[u].y = fmaf(args.beta2, o[u].y, sum[k + (MODE == kStats ? 1 : 0)]);
-              o[u].z = fmaf(args.beta2, o[u].z, sum[k + (MODE == kStats ? 2 : 0)]);
-              o[u].w = fmaf(args.beta2, o[u].w, sum[k + (MODE == kStats ? 3 : 0)]);
-              row[u] = o[u];
+              for (int u = 0; u < 8; ++u) o[8 * gq + u] = row[u];
+            }
+          }
+#pragma unroll
+          for (int gq = 0; gq < NG; ++gq) {
+            const int cb = j0 + (c0 + gq) * 32;
+            if (r < S && cb < S) {
+              float4* row = reinterpret_cast<float4*>(C + (size_t)r * S + cb);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const int k = MODE == kStats ? 32 * (c0 + gq) + 4 * u : 0;
+                float4 v = o[8 * gq + u];
+                v.x = fmaf(args.beta2, v.x, sum[k]);
+                v.y = fmaf(args.beta2, v.y, sum[k + (MODE == kStats ? 1 : 0)]);
+                v.z = fmaf(args.beta2, v.z, sum[k + (MODE == kStats ? 2 : 0)]);
+                v.w = fmaf(args.beta2, v.w, sum[k + (MODE == kStats ? 3 : 0)]);
+                row[u] = v;
+              }
             }
           }
         }
@@ -509,7 +537,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 1) tc::tmem_dealloc(tmem, 256);
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // K1: gradients -> blocked, zero-padded bf16 planes.  grid: x = 2048-element
@@ -683,7 +711,8 @@ cudaError_t launch_stats_tc(const TcMaps& maps, const BlockDesc* blocks, const i
   a.blocks = blocks; a.flags = flags; a.nblk = nblk; a.nmat = nmat; a.S = S;
   a.planes_g = planes_g; a.beta2 = beta2; a.stats = stats; a.err = err; a.stall = stall;
   const int T = (S + kTM - 1) / kTM;
-  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2), smem_bytes(planes_g, S <= kTM ? 0 : planes_g, planes_g == 1),
+  return launch_mode<kStats>(nblk * 2 * (T * (T + 1) / 2),
+                             smem_bytes(planes_g, S <= kTM ? 0 : planes_g, stats_cstage(planes_g, S)),
                              maps, a, s);
 }
 
