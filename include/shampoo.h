@@ -370,9 +370,8 @@ shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int bat
  * GPU (from other streams or host threads) race; serialise them.  Every call
  * looks up the work space's device address on the current device (nothing is
  * kept between calls, so a device reset cannot leave a stale address); the
- * first lookup in a process may load the library's device code, so make the
- * first call before any stream capture begins.  Synchronises with the host
- * while it runs.
+ * first lookup in a process may load the library's device code.
+ * Synchronises with the host while it runs.
  */
 shampoo_status shampoo_batched_inverse_root_noalloc(const float* A, float* X, int batch, int n,
                                                     int p, float eps, double tol, int max_iters,

@@ -22,8 +22,7 @@
 //    (cudaGetSymbolAddress with that device current) instead of keeping it:
 //    after a device reset, or under another driver context, the array can sit
 //    at another address, and a kept one would point at freed memory.  The
-//    first lookup in a process may load the library's device code, so make
-//    the first call before any stream capture begins.
+//    first lookup in a process may load the library's device code.
 #include <string>
 
 #include "../../include/shampoo.h"
