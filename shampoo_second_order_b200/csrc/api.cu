@@ -444,6 +444,20 @@ bool encode_planes(CUtensorMap* m, void* base, int S, int64_t depth, int box_x, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The gradient planes [planes][nblk][S][S] bf16 as a 4-D tensor (col, row,
+// block, plane) whose boxes hold `planes` planes of one block's panel.
+bool encode_planes4(CUtensorMap* m, void* base, int S, int64_t nblk, int planes, int box_x, int box_y) {
+  auto fn = encode_fn();
+  if (!fn || nblk < 1) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)S, (cuuint64_t)S, (cuuint64_t)nblk, (cuuint64_t)planes};
+  cuuint64_t strides[3] = {(cuuint64_t)S * 2, (cuuint64_t)S * S * 2, (cuuint64_t)nblk * S * S * 2};
+  cuuint32_t box[4] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1, (cuuint32_t)planes};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr const char* kTimeoutMsg =
     "a tensor-core kernel timed out waiting on its pipeline and aborted; the optimizer state of this "
     "context is no longer valid (destroy it and start a new one)";
@@ -864,6 +878,8 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   if (nblk64 &&
       !(encode_planes(&ctx->maps.gk, ctx->gblk, b, ctx->planes_g * nblk64, 64, 128) &&
         encode_planes(&ctx->maps.gmn, ctx->gblk, b, ctx->planes_g * nblk64, 64, 64) &&
+        encode_planes4(&ctx->maps.gk4, ctx->gblk, b, nblk64, ctx->planes_g, 64, 128) &&
+        encode_planes4(&ctx->maps.gmn4, ctx->gblk, b, nblk64, ctx->planes_g, 64, 64) &&
         encode_planes(&ctx->maps.rk, ctx->rplanes, b, 2 * (int64_t)ctx->nmat, 64, 128) &&
         encode_planes(&ctx->maps.ymn, ctx->yplanes, b, 2 * nblk64, 64, 64) &&
         encode_planes(&ctx->maps.ck, ctx->stats, b, ctx->nmat, 32, 128, true))) {

@@ -59,6 +59,9 @@ struct NewtonMat {
 //  ck   statistics fp32 [nmat][S][S], box 32 x 128 (the update's read-modify-write)
 struct TcMaps {
   CUtensorMap gk, gmn, rk, ymn, ck;
+  // the gradient planes as [plane][block][row][col], for boxes that carry
+  // both planes of a panel (the statistics)
+  CUtensorMap gk4, gmn4;
 };
 
 // ---------------- tensor-core kernels (k_tc.cu) ----------------

@@ -237,12 +237,27 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         const bool diag = (MODE == kStats) && i0 == j0;
         tc::mbar_expect_tx(&full[s], diag ? nA * kBoxBytes : stage_bytes);
         const int k0 = kt * kBKe;
+        if (MODE == kStats) {
+          // one 4-D box carries both planes of a panel (h and m of fp32
+          // gradients): K-major [plane][128 rows][64 K], or MN-major in two
+          // 64-wide halves [half][plane][64 K][64]
+          if (isR) {
+            const int hb = nA * kBoxBytes / 2;
+            tc::tma_load_4d(st, mA, &full[s], i0, k0, blk, 0);
+            tc::tma_load_4d(st + hb, mA, &full[s], i0 + 64, k0, blk, 0);
+            if (!diag) {
+              tc::tma_load_4d(st + nA * kBoxBytes, mB, &full[s], j0, k0, blk, 0);
+              tc::tma_load_4d(st + nA * kBoxBytes + hb, mB, &full[s], j0 + 64, k0, blk, 0);
+            }
+          } else {
+            tc::tma_load_4d(st, mA, &full[s], k0, i0, blk, 0);
+            if (!diag) tc::tma_load_4d(st + nA * kBoxBytes, mB, &full[s], k0, j0, blk, 0);
+          }
+          continue;
+        }
         for (int pa = 0; pa < nA; ++pa) {
           uint8_t* dst = st + pa * kBoxBytes;
-          if (MODE == kStats && isR) {          // A(i, k) = G[k][i]: two 64-wide boxes along i
-            tc::tma_load_3d(dst, mA, &full[s], i0, k0, pa * args.nblk + blk);
-            tc::tma_load_3d(dst + kBoxBytes / 2, mA, &full[s], i0 + 64, k0, pa * args.nblk + blk);
-          } else if (MODE == kApplyP) {         // A = L^{-1/p} planes
+          if (MODE == kApplyP) {                // A = L^{-1/p} planes
             tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nmat + 2 * blk);
           } else {                              // A = G rows
             tc::tma_load_3d(dst, mA, &full[s], k0, i0, pa * args.nblk + blk);
@@ -250,12 +265,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
         }
         for (int pb = 0; pb < nB && !diag; ++pb) {
           uint8_t* dst = st + (nA + pb) * kBoxBytes;
-          if (MODE == kStats && isR) {
-            tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
-            tc::tma_load_3d(dst + kBoxBytes / 2, mB, &full[s], j0 + 64, k0, pb * args.nblk + blk);
-          } else if (MODE == kStats) {
-            tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nblk + blk);
-          } else if (MODE == kApplyY) {         // B(k, j) = R^{-1/p}[j][k] (symmetric)
+          if (MODE == kApplyY) {                // B(k, j) = R^{-1/p}[j][k] (symmetric)
             tc::tma_load_3d(dst, mB, &full[s], k0, j0, pb * args.nmat + 2 * blk + 1);
           } else {                              // B(k, j) = Y[k][j], MN-major
             tc::tma_load_3d(dst, mB, &full[s], j0, k0, pb * args.nblk + blk);
@@ -313,6 +323,30 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
           // statistics: a stage's small split products (hm mh mm) go into
           // the accumulator before its large h h products, while the running
           // sum is still small, so their truncation costs less
+          if (MODE == kStats && npass == 4) {
+            // fp32 gradients: the 16 MMAs of the stage from descriptors made
+            // once per stage (a single thread issues them back to back; the
+            // generic loop below costs it about as long as the MMAs take)
+            // planes: K-major one box apart; MN-major half a box apart, with
+            // the second 64-wide half of both planes one box further
+            const uint64_t tmpl = a_mn ? tc::smem_desc(0, kBoxBytes, 1024) : tc::smem_desc(0, 16, 1024);
+            const uint32_t step = a_mn ? 128u : 2u;   // one 16-deep slice, in 16-byte units
+            const uint32_t po = a_mn ? kBoxBytes / 2 : kBoxBytes;
+            const uint64_t ah = tmpl + (st >> 4), am = tmpl + ((st + po) >> 4);
+            const uint64_t bh = diag ? ah : tmpl + ((st + 2 * kBoxBytes) >> 4);
+            const uint64_t bm = diag ? am : tmpl + ((st + 2 * kBoxBytes + po) >> 4);
+            const uint32_t first = (kt - c0) != 0;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(dt, ah + step * kk, bm + step * kk, idesc, first | kk);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(dt, am + step * kk, bh + step * kk, idesc, 1u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(dt, am + step * kk, bm + step * kk, idesc, 1u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc::mma_bf16(dt, ah + step * kk, bh + step * kk, idesc, 1u);
+            tc::mma_commit(&empty[s]);
+            continue;
+          }
           for (int qq = 0; qq < npass; ++qq) {
             const int q = (MODE == kStats && kCorrFirst) ? (qq + 1 < npass ? qq + 1 : 0) : qq;
 #pragma unroll
@@ -667,7 +701,10 @@ cudaError_t launch_mode(int ntiles, size_t smem, const TcMaps& maps, const TcArg
     configured = true;
   }
   const int grid = ntiles < sm_count() ? ntiles : sm_count();
-  tc_gemm_kernel<MODE><<<grid, 192, smem, s>>>(maps.gk, maps.gmn, maps.rk, maps.ymn, maps.ck, a, ntiles);
+  // the statistics load both gradient planes of a panel in one 4-D box
+  tc_gemm_kernel<MODE><<<grid, 192, smem, s>>>(MODE == kStats ? maps.gk4 : maps.gk,
+                                               MODE == kStats ? maps.gmn4 : maps.gmn, maps.rk, maps.ymn,
+                                               maps.ck, a, ntiles);
   return cudaGetLastError();
 }
 
