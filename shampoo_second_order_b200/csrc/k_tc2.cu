@@ -24,8 +24,10 @@
 //
 // (The statistics stay on the single-CTA kernel: their two-level
 // accumulation keeps a running sum of 128 columns per thread in registers,
-// which 256-column pair tiles cannot hold, and 256 x 128 pair tiles, which
-// can, measured 13% slower than single-CTA 128 x 128 tiles at b = 1024.)  Every wait is bounded; a give-up
+// which 256-column pair tiles cannot hold.  256 x 128 pair tiles, which can,
+// measured 7-13% slower than single-CTA 128 x 128 tiles at b = 1024: pairing
+// the upper-triangle tiles of a column panel computes 11% extra tiles there,
+// more than the pair saves.)  Every wait is bounded; a give-up
 // sets the error word and both CTAs' abort flags, each producer lets its own
 // loads land, the MMA issuer lets its MMAs land, and the pair meets at a
 // cluster barrier before freeing TMEM and returning.
