@@ -54,11 +54,12 @@ UNIT = "TFLOP/s"
 # workload, mode or kernel until measured there.
 TRAFFIC_PER_LAUNCH = {
     # the statistics GEMM (single-CTA 128x128 tiles, 2-term split with four
-    # products, two-level accumulation over four TMEM accumulators): 230.7 MB
-    # for the 20 blocks of Transformer-big layer 0 (ncu, one launch, `python -m
+    # products, two-level accumulation over four TMEM accumulators, both
+    # gradient planes of a panel per TMA box): 231.5 MB for the 20 blocks of
+    # Transformer-big layer 0 (ncu, one launch, `python -m
     # shampoo_second_order_b200.run_steps`), scaled by the block count to the
     # 272 identical 1024 x 1024 blocks of a full launch
-    ("transformer_big_b1024", "stats_tc"): 230749696 * 272 // 20,
+    ("transformer_big_b1024", "stats_tc"): 231501056 * 272 // 20,
 }
 
 

@@ -165,6 +165,9 @@ struct shampoo_ctx {
   TcMaps maps{};
   int planes_g = 1;
   int* d_err = nullptr;
+  // pointer tables as last uploaded to d_gptr / d_wptr
+  std::vector<const void*> sent_gptr;
+  std::vector<float*> sent_wptr;
   std::vector<const void*> gathered_from;   // gradient pointers of the last gather
   std::vector<const void*> stats_from;      // gradient pointers of the last update_stats
   double* d2 = nullptr;   // [nparams] ||D||^2 of the graft target
@@ -403,14 +406,21 @@ shampoo_status set_pointers(shampoo_ctx* ctx, const void* const* grads, float* c
   if (!grads) return fail(ctx, SHAMPOO_EINVAL, "grads is NULL");
   for (int i = 0; i < ctx->nparams; ++i)
     if (!grads[i]) return fail(ctx, SHAMPOO_EINVAL, "grads[" + std::to_string(i) + "] is NULL");
-  // pageable source: staged by the driver before the call returns
-  CK(cudaMemcpyAsync(ctx->d_gptr, grads, ctx->nparams * sizeof(void*), cudaMemcpyHostToDevice,
-                     ctx->stream));
+  // pageable source: staged by the driver before the call returns; tables
+  // that equal the last ones uploaded are not sent again
+  if (!std::equal(grads, grads + ctx->nparams, ctx->sent_gptr.begin(), ctx->sent_gptr.end())) {
+    CK(cudaMemcpyAsync(ctx->d_gptr, grads, ctx->nparams * sizeof(void*), cudaMemcpyHostToDevice,
+                       ctx->stream));
+    ctx->sent_gptr.assign(grads, grads + ctx->nparams);
+  }
   if (params) {
     for (int i = 0; i < ctx->nparams; ++i)
       if (!params[i]) return fail(ctx, SHAMPOO_EINVAL, "params[" + std::to_string(i) + "] is NULL");
-    CK(cudaMemcpyAsync(ctx->d_wptr, params, ctx->nparams * sizeof(float*), cudaMemcpyHostToDevice,
-                       ctx->stream));
+    if (!std::equal(params, params + ctx->nparams, ctx->sent_wptr.begin(), ctx->sent_wptr.end())) {
+      CK(cudaMemcpyAsync(ctx->d_wptr, params, ctx->nparams * sizeof(float*), cudaMemcpyHostToDevice,
+                         ctx->stream));
+      ctx->sent_wptr.assign(params, params + ctx->nparams);
+    }
   }
   return SHAMPOO_OK;
 }

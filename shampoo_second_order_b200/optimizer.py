@@ -20,6 +20,7 @@ class Shampoo:
                  grad_dtype="f32", stream=None):
         import torch
         self.shapes = [tuple(s) for s in shapes]
+        self._numel = [int(np.prod(s)) for s in self.shapes]   # checked on every call
         self.block_size = int(block_size)
         if stream is None:
             stream = torch.cuda.current_stream()
@@ -29,10 +30,10 @@ class Shampoo:
         self.ctx = L.shampoo_create(self.shapes, block_size, beta2, eps, p, graft, momentum, dt, handle)
 
     def _check_tensors(self, ts, what):
-        if len(ts) != len(self.shapes):
-            raise ValueError(f"expected {len(self.shapes)} {what}, got {len(ts)}")
-        for t, s in zip(ts, self.shapes):
-            if not (t.is_cuda and t.is_contiguous()) or t.numel() != int(np.prod(s)):
+        if len(ts) != len(self._numel):
+            raise ValueError(f"expected {len(self._numel)} {what}, got {len(ts)}")
+        for t, k in zip(ts, self._numel):
+            if t.numel() != k or not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{what} must be contiguous CUDA tensors of the given shapes")
 
     def update_stats(self, grads):
