@@ -569,6 +569,31 @@ cudaError_t batched_pool(cudaMemPool_t* out) {
   return cudaSuccess;
 }
 
+// The pinned counters and the two events a batched root call polls with, per
+// host thread and device, made on the thread's first call there and kept:
+// pinning host memory and freeing it (which synchronises the device) on
+// every call cost more than the call's own host work.
+cudaError_t batched_host_state(int** h_count, cudaEvent_t* ev) {
+  struct State {
+    int* h = nullptr;
+    cudaEvent_t ev[2] = {nullptr, nullptr};
+  };
+  thread_local State st[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  State& x = st[dev];
+  if (!x.h && (e = cudaMallocHost(&x.h, 3 * sizeof(int))) != cudaSuccess) return e;
+  for (auto& v : x.ev)
+    if (!v && (e = cudaEventCreateWithFlags(&v, cudaEventDisableTiming)) != cudaSuccess) return e;
+  x.h[0] = x.h[1] = x.h[2] = 0;
+  *h_count = x.h;
+  ev[0] = x.ev[0];
+  ev[1] = x.ev[1];
+  return cudaSuccess;
+}
+
 // ---------------- asynchronous root pipeline ----------------
 
 // One root job, on the root thread: Newton on the statistics copy into the
@@ -1338,9 +1363,7 @@ shampoo_status shampoo_batched_inverse_root_ex(const float* A, float* X, int bat
     res = fail(ctx, SHAMPOO_ENOMEM, std::string("work space: ") + cudaGetErrorString(e));
     goto done;
   }
-  if ((e = cudaMallocHost(&ctx->h_count, 3 * sizeof(int))) != cudaSuccess ||
-      (e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming)) != cudaSuccess ||
-      (e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming)) != cudaSuccess ||
+  if ((e = batched_host_state(&ctx->h_count, ctx->ev)) != cudaSuccess ||
       (e = dalloc(ctx, &ctx->d_err, 1)) != cudaSuccess ||
       (e = cudaMemsetAsync(ctx->d_err, 0, sizeof(int), st)) != cudaSuccess) {
     res = cuda_fail(ctx, e, "set-up");
@@ -1370,10 +1393,7 @@ done:
   for (void* q : ctx->allocs) cudaFreeAsync(q, st);   // back to the pool, in stream order
   ctx->allocs.clear();
   cudaStreamSynchronize(st);
-  if (ctx->h_count) cudaFreeHost(ctx->h_count);
-  ctx->h_count = nullptr;
-  for (auto& ev : ctx->ev)
-    if (ev) cudaEventDestroy(ev);
+  ctx->h_count = nullptr;   // this thread's, kept for its next call
   ctx->ev[0] = ctx->ev[1] = nullptr;
   if (res != SHAMPOO_OK) g_create_err = ctx->err;
   return res;
