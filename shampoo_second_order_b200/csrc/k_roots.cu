@@ -794,7 +794,11 @@ void launch_newton_init(const float* A, int64_t a_stride, int lda, int upper, co
 }
 
 void launch_newton_lanczos(const NewtonMat* mats, int nm, int S, NewtonWork w, cudaStream_t s) {
-  const int threads = S <= 128 ? 128 : (S <= 256 ? 256 : 512);   // one warp per row at a time
+  // Each warp streams two rows of the statistic at a time, so a matvec takes
+  // n / (2 x warps) dependent passes: small sides use fewer warps per matrix
+  // to fit more matrices on the GPU, unless there are few matrices, where
+  // every pass is latency and more warps per matrix shorten the chain.
+  const int threads = (S <= 128 && nm > 296) ? 128 : ((S <= 256 && nm > 296) ? 256 : 512);
   newton_lanczos_kernel<<<nm, threads, 0, s>>>(mats, S, w);
 }
 
