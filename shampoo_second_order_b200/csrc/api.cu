@@ -589,7 +589,9 @@ cudaError_t batched_pool(cudaMemPool_t* out) {
 // The pinned counters and the two events a batched root call polls with, per
 // host thread and device, made on the thread's first call there and kept:
 // pinning host memory and freeing it (which synchronises the device) on
-// every call cost more than the call's own host work.
+// every call cost more than the call's own host work.  Each call checks that
+// they still belong to a live context (a device reset frees both) and makes
+// them again if not.
 cudaError_t batched_host_state(int** h_count, cudaEvent_t* ev) {
   struct State {
     int* h = nullptr;
@@ -601,6 +603,21 @@ cudaError_t batched_host_state(int** h_count, cudaEvent_t* ev) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   State& x = st[dev];
+  if (x.h) {
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, x.h) != cudaSuccess || at.type != cudaMemoryTypeHost) {
+      cudaGetLastError();   // clear the lookup's error
+      x.h = nullptr;        // released with its context
+    }
+  }
+  for (auto& v : x.ev) {
+    if (!v) continue;
+    const cudaError_t q = cudaEventQuery(v);
+    if (q != cudaSuccess && q != cudaErrorNotReady) {
+      cudaGetLastError();
+      v = nullptr;          // destroyed with its context
+    }
+  }
   if (!x.h && (e = cudaMallocHost(&x.h, 3 * sizeof(int))) != cudaSuccess) return e;
   for (auto& v : x.ev)
     if (!v && (e = cudaEventCreateWithFlags(&v, cudaEventDisableTiming)) != cudaSuccess) return e;
