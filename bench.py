@@ -203,6 +203,19 @@ def job_tflops(flops_per_rank, world, job_ms):
 # ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
+def flat_views(flat, shapes):
+    """Contiguous per-parameter views of a flat 1-D tensor that holds the
+    parameters back to back, row-major, in the order of `shapes`."""
+    out, o = [], 0
+    for sh in shapes:
+        n = int(np.prod(sh))
+        out.append(flat[o:o + n].view(*sh))
+        o += n
+    if o != flat.numel():
+        raise ValueError(f"flat buffer holds {flat.numel()} elements, the shapes {o}")
+    return out
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -884,22 +897,19 @@ def main():
     # device-resident number.
     e2e = None
     if not args.no_e2e:
-        sizes = [int(np.prod(w.shape)) for w in W0]
-        offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
-
-        def views(flat):
-            return [flat[int(offs[i]):int(offs[i + 1])].view(W0[i].shape) for i in range(len(W0))]
+        shapes_w = [tuple(w.shape) for w in W0]
+        total = sum(int(np.prod(sh)) for sh in shapes_w)
         pin_g = []
         for gs in host_grads[:2]:
-            flat = torch.empty(int(offs[-1]), dtype=gdt).pin_memory()
-            for v, g in zip(views(flat), gs):
+            flat = torch.empty(total, dtype=gdt).pin_memory()
+            for v, g in zip(flat_views(flat, shapes_w), gs):
                 v.copy_(torch.from_numpy(g).to(gdt))
             pin_g.append(flat)
-        pin_w = [torch.empty(int(offs[-1]), dtype=torch.float32).pin_memory() for _ in range(2)]
-        dG_flat = [torch.empty(int(offs[-1]), dtype=gdt, device=dev) for _ in range(2)]
-        dG = [views(f) for f in dG_flat]
-        snap_flat = [torch.empty(int(offs[-1]), dtype=torch.float32, device=dev) for _ in range(2)]
-        snap = [views(f) for f in snap_flat]
+        pin_w = [torch.empty(total, dtype=torch.float32).pin_memory() for _ in range(2)]
+        dG_flat = [torch.empty(total, dtype=gdt, device=dev) for _ in range(2)]
+        dG = [flat_views(f, shapes_w) for f in dG_flat]
+        snap_flat = [torch.empty(total, dtype=torch.float32, device=dev) for _ in range(2)]
+        snap = [flat_views(f, shapes_w) for f in snap_flat]
         h2d = pin_g[0].numel() * pin_g[0].element_size()
         d2h = pin_w[0].numel() * 4
         up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)

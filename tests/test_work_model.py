@@ -123,3 +123,27 @@ def test_both_arms_credit_the_same_step_work():
         bench.stats_flops(c) + bench.apply_flops(c) + roots / 100)
     one = dict(wl.CONFIGS["single_64x32"], right_only=[0])
     assert bench.credit_iters(one, 6) == [0, 6]
+
+
+def test_end_to_end_buffers_are_the_parameters_back_to_back():
+    """The end-to-end loop uploads each step's gradients as one flat buffer and
+    hands the optimizer per-parameter views of it: the views must be
+    contiguous, shaped like the parameters, cover the buffer exactly in order,
+    and the bytes per step must be the parameters' bytes."""
+    import numpy as np
+    import torch
+    shapes = [s if len(s) == 2 else (s[0],) for s in wl.CONFIGS["resnet50_b128"]["shapes"][:12]]
+    total = sum(int(np.prod(s)) for s in shapes)
+    flat = torch.arange(total, dtype=torch.float32)
+    vs = bench.flat_views(flat, shapes)
+    assert [tuple(v.shape) for v in vs] == [tuple(s) for s in shapes]
+    assert all(v.is_contiguous() for v in vs)
+    o = 0
+    for v in vs:   # element k of view i is element offs[i] + k of the buffer
+        assert float(v.reshape(-1)[0]) == o and float(v.reshape(-1)[-1]) == o + v.numel() - 1
+        o += v.numel()
+    assert o == total == flat.numel()
+    assert flat.numel() * 4 == sum(int(np.prod(s)) * 4 for s in shapes)
+    import pytest
+    with pytest.raises(ValueError):
+        bench.flat_views(torch.zeros(total + 1), shapes)
