@@ -42,10 +42,6 @@ constexpr int kBoxBytes = kTM * kBKe * 2;   // 16 KB: one operand plane per stag
 #define SHAMPOO_STATS_CHUNK_STAGES 1
 #endif
 constexpr int kChunkStages = SHAMPOO_STATS_CHUNK_STAGES;   // statistics: K stages per accumulation chunk
-#ifndef SHAMPOO_STATS_CORR_FIRST
-#define SHAMPOO_STATS_CORR_FIRST 1
-#endif
-constexpr bool kCorrFirst = SHAMPOO_STATS_CORR_FIRST != 0;
 // TMEM accumulators of the statistics GEMM (4 x 128 columns): the MMA issuer
 // may run three K chunks ahead of the epilogue, which stops draining TMEM
 // while it read-modify-writes a finished tile
@@ -160,9 +156,7 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
   if (MODE == kStats && g1) {
     npass = 1; pas = 0; pbs = 0;                          // g g
   } else if (MODE == kStats) {
-    npass = 4;                                            // hh hm mh mm
-    pas = (0u) | (0u << 2) | (1u << 4) | (1u << 6);
-    pbs = (0u) | (1u << 2) | (0u << 4) | (1u << 6);
+    npass = 4; pas = 0; pbs = 0;                          // hm mh mm hh, issued explicitly
   } else if (MODE == kApplyY && g1) {
     npass = 2; pas = 0; pbs = (1u << 2);                  // g R_h, g R_l
   } else {
@@ -324,11 +318,10 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
           // the accumulator before its large h h products, while the running
           // sum is still small, so their truncation costs less
           if (MODE == kStats && npass == 4) {
-            // fp32 gradients: the 16 MMAs of the stage from descriptors made
-            // once per stage (a single thread issues them back to back; the
-            // generic loop below costs it about as long as the MMAs take)
-            // planes: K-major one box apart; MN-major half a box apart, with
-            // the second 64-wide half of both planes one box further
+            // fp32 gradients: the stage's 16 MMAs, h m, m h, m m, then h h,
+            // from descriptors made once per stage.  Planes: K-major one box
+            // apart; MN-major half a box apart, with the second 64-wide half
+            // of both planes one box further
             const uint64_t tmpl = a_mn ? tc::smem_desc(0, kBoxBytes, 1024) : tc::smem_desc(0, 16, 1024);
             const uint32_t step = a_mn ? 128u : 2u;   // one 16-deep slice, in 16-byte units
             const uint32_t po = a_mn ? kBoxBytes / 2 : kBoxBytes;
@@ -348,11 +341,10 @@ __global__ void __launch_bounds__(192, 1) tc_gemm_kernel(const __grid_constant__
             continue;
           }
           for (int qq = 0; qq < npass; ++qq) {
-            const int q = (MODE == kStats && kCorrFirst) ? (qq + 1 < npass ? qq + 1 : 0) : qq;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const int pa = (pas >> (2 * q)) & 3;
-              const int pb = (pbs >> (2 * q)) & 3;
+              const int pa = (pas >> (2 * qq)) & 3;
+              const int pb = (pbs >> (2 * qq)) & 3;
               const uint32_t sa = st + pa * kBoxBytes;
               const uint32_t sb = st + (diag ? pb : nA + pb) * kBoxBytes;
               const uint64_t da = a_mn ? tc::smem_desc(sa + kk * 2048, 8192, 1024)
