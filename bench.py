@@ -57,8 +57,9 @@ TRAFFIC_PER_LAUNCH = {
     # products, two-level accumulation over four TMEM accumulators, both
     # gradient planes of a panel per TMA box): 231.5 MB for the 20 blocks of
     # Transformer-big layer 0 (ncu, one launch, `python -m
-    # shampoo_second_order_b200.run_steps`), scaled by the block count to the
-    # 272 identical 1024 x 1024 blocks of a full launch
+    # shampoo_second_order_b200.run_steps`, kernel of d53cb9c; the later edits
+    # of k_tc.cu left this path's loads and stores unchanged), scaled by the
+    # block count to the 272 identical 1024 x 1024 blocks of a full launch
     ("transformer_big_b1024", "stats_tc"): 231501056 * 272 // 20,
 }
 
