@@ -128,13 +128,6 @@ struct shampoo_ctx {
   // events
   cudaStream_t aux = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_mid = nullptr, ev_join = nullptr;
-  // update_stats' work on `aux` (1-D check, accumulator, 1-D statistics) is
-  // joined into `stream` by the first later call that reads what it writes,
-  // not at the end of update_stats: while the statistics GEMM holds every
-  // SM's registers it cannot start, and it then runs beside the next call's
-  // GEMMs instead of after the statistics
-  cudaEvent_t ev_stats_aux = nullptr;
-  bool aux_pending = false;
   int nparams = 0, b = 0, S = 0, p = 4, graft = 1, bf16 = 0;
   float beta2 = 1.f, eps = 1e-6f, mu = 0.f;
   double tol = 1e-6;
@@ -501,16 +494,6 @@ shampoo_status poll_kernel_error(shampoo_ctx* ctx) {
   return SHAMPOO_OK;
 }
 
-// Make `stream` wait for update_stats' work on the auxiliary stream, if it
-// has not yet: every call that reads the flags, the accumulator, its norms
-// or the 1-D statistics calls this first.
-shampoo_status join_aux(shampoo_ctx* ctx) {
-  if (!ctx->aux_pending) return SHAMPOO_OK;
-  CK(cudaStreamWaitEvent(ctx->stream, ctx->ev_stats_aux, 0));
-  ctx->aux_pending = false;
-  return SHAMPOO_OK;
-}
-
 // Gather the 2-D gradients into the blocked bf16 planes unless the planes
 // already hold these very gradient pointers from this step's update_stats.
 shampoo_status gather(shampoo_ctx* ctx, const void* const* grads, bool force) {
@@ -782,7 +765,6 @@ void shampoo_destroy(shampoo_ctx* ctx) {
   if (ctx->ev_fork) cudaEventDestroy(ctx->ev_fork);
   if (ctx->ev_mid) cudaEventDestroy(ctx->ev_mid);
   if (ctx->ev_join) cudaEventDestroy(ctx->ev_join);
-  if (ctx->ev_stats_aux) cudaEventDestroy(ctx->ev_stats_aux);
   cudaStreamSynchronize(ctx->stream);
   for (void* q : ctx->allocs) cudaFree(q);
   if (ctx->h_count) cudaFreeHost(ctx->h_count);
@@ -926,7 +908,6 @@ shampoo_status shampoo_create(shampoo_ctx** out, int nparams, const int64_t* sha
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_mid, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_join, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_stats_aux, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[0], cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev[1], cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->stats, 0, ctx->nmat * slot * sizeof(float), ctx->stream);
@@ -965,8 +946,6 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   shampoo_status st = poll_kernel_error(ctx);
   if (st != SHAMPOO_OK) return st;
-  st = join_aux(ctx);   // the previous call's accumulator pass reads the flags and pointers reset next
-  if (st != SHAMPOO_OK) return st;
   st = set_pointers(ctx, grads, nullptr);
   if (st != SHAMPOO_OK) return st;
   cudaStream_t s = ctx->stream, x = ctx->aux;
@@ -1003,8 +982,7 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
       launch_stats_segments(ctx->d_segs, nseg, 2 * nblk, ctx->d_gptr, ctx->bf16, ctx->flags,
                             ctx->beta2, ctx->stats, ctx->S, x);
     });
-  CK(cudaEventRecord(ctx->ev_stats_aux, x));
-  ctx->aux_pending = true;
+  CK(cudaEventRecord(ctx->ev_join, x));
   ctx->stats_from.assign(grads, grads + ctx->nparams);
   if (nblk) {
     cudaError_t e = cudaSuccess;
@@ -1015,6 +993,7 @@ shampoo_status shampoo_update_stats(shampoo_ctx* ctx, const void* const* grads) 
     ctx->stall_next_stats = 0;
     if (e != cudaSuccess) return cuda_fail(ctx, e, "stats_tc");
   }
+  CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
   CK(cudaGetLastError());
   ctx->stats_done = true;
   return SHAMPOO_OK;
@@ -1025,10 +1004,6 @@ shampoo_status shampoo_compute_roots(shampoo_ctx* ctx) {
   int nf = 0, mi = 0;
   if (!ctx->stats_done) return fail(ctx, SHAMPOO_ESTATE, "compute_roots before update_stats");
   if (job_in_flight(ctx)) return fail(ctx, SHAMPOO_EBUSY, "an asynchronous root job is in flight");
-  {   // the 1-D statistics come from the auxiliary stream
-    const shampoo_status js = join_aux(ctx);
-    if (js != SHAMPOO_OK) return js;
-  }
   {   // statistics left by an aborted GEMM are not rooted: this call synchronises anyway
     const shampoo_status ks = check_kernel_error(ctx);
     if (ks != SHAMPOO_OK) return ks;
@@ -1089,10 +1064,6 @@ shampoo_status shampoo_compute_roots_async(shampoo_ctx* ctx) {
     ctx->nw.qs = ctx->oz_slices;
   }
   // the statistics as they stand after every call so far
-  {
-    const shampoo_status js = join_aux(ctx);
-    if (js != SHAMPOO_OK) return js;
-  }
   const size_t n = (size_t)ctx->nmat * ctx->S * ctx->S;
   CK(cudaMemcpyAsync(ctx->stats_snap, ctx->stats, n * sizeof(float), cudaMemcpyDeviceToDevice, ctx->stream));
   CK(cudaEventRecord(ctx->ev_submit, ctx->stream));
@@ -1127,12 +1098,6 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
   }
   if (!ctx->roots_done) return fail(ctx, SHAMPOO_ESTATE, "apply before compute_roots");
   if (!params) return fail(ctx, SHAMPOO_EINVAL, "params is NULL");
-  bool same = ctx->stats_from.size() == (size_t)ctx->nparams;
-  for (int i = 0; same && i < ctx->nparams; ++i) same = ctx->stats_from[i] == grads[i];
-  if (!same) {   // other gradients: the pointer table and the flags that the accumulator pass reads change
-    const shampoo_status js = join_aux(ctx);
-    if (js != SHAMPOO_OK) return js;
-  }
   shampoo_status st = set_pointers(ctx, grads, params);
   if (st != SHAMPOO_OK) return st;
   cudaStream_t s = ctx->stream;
@@ -1150,6 +1115,15 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
                                    ctx->aux);
     });
     CK(cudaEventRecord(ctx->ev_join, ctx->aux));
+  }
+  bool same = ctx->stats_from.size() == (size_t)ctx->nparams;
+  for (int i = 0; same && i < ctx->nparams; ++i) same = ctx->stats_from[i] == grads[i];
+  if (ctx->graft && !same) {   // ||D||^2 of these gradients against the current a
+    CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), s));
+    run(pr, "dnorm", s, [&] {
+      launch_dnorm(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->a,
+                   ctx->eps, ctx->d2, s);
+    });
   }
   if (nblk) {
     shampoo_status gs = gather(ctx, grads, false);
@@ -1171,17 +1145,6 @@ shampoo_status shampoo_apply(shampoo_ctx* ctx, float* const* params, const void*
                                    ctx->S, ctx->P, ctx->p2, ctx->d_err, s);
     });
     if (e != cudaSuccess) return cuda_fail(ctx, e, "apply_p_tc");
-  }
-  {   // the accumulator and its norms (the statistics' auxiliary work) before the update
-    const shampoo_status js = join_aux(ctx);
-    if (js != SHAMPOO_OK) return js;
-  }
-  if (ctx->graft && !same) {   // ||D||^2 of these gradients against the current a
-    CK(cudaMemsetAsync(ctx->d2, 0, ctx->nparams * sizeof(double), s));
-    run(pr, "dnorm", s, [&] {
-      launch_dnorm(ctx->d_chunks, nch, ctx->d_params, ctx->d_gptr, ctx->bf16, ctx->flags, ctx->a,
-                   ctx->eps, ctx->d2, s);
-    });
   }
   if (nseg) CK(cudaStreamWaitEvent(s, ctx->ev_join, 0));
   run(pr, "update", s, [&] {
@@ -1206,10 +1169,6 @@ shampoo_status shampoo_root_status(shampoo_ctx* ctx, int* n_not_converged, int* 
 shampoo_status shampoo_nonfinite_status(shampoo_ctx* ctx, int* n_params_skipped) {
   if (!ctx) return fail(nullptr, SHAMPOO_EINVAL, "ctx is NULL");
   if (!n_params_skipped) return fail(ctx, SHAMPOO_EINVAL, "n_params_skipped is NULL");
-  {   // the 1-D check runs on the auxiliary stream
-    const shampoo_status js = join_aux(ctx);
-    if (js != SHAMPOO_OK) return js;
-  }
   std::vector<int> f(ctx->nparams);
   CK(cudaMemcpyAsync(f.data(), ctx->flags, ctx->nparams * sizeof(int), cudaMemcpyDeviceToHost,
                      ctx->stream));
@@ -1330,10 +1289,6 @@ shampoo_status shampoo_read_matrix(shampoo_ctx* ctx, int which, int index, float
     return fail(ctx, SHAMPOO_EINVAL, "bad which / index / dst");
   const size_t slot = (size_t)ctx->S * ctx->S;
   const float* src = (which == 0 ? ctx->stats : ctx->roots) + slot * index;
-  {
-    const shampoo_status js = join_aux(ctx);
-    if (js != SHAMPOO_OK) return js;
-  }
   std::vector<float> h(slot);
   CK(cudaMemcpyAsync(h.data(), src, slot * sizeof(float), cudaMemcpyDeviceToHost, ctx->stream));
   CK(cudaStreamSynchronize(ctx->stream));
