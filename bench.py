@@ -712,6 +712,88 @@ def shard_bench(args, cfg, rank, world, local):
         newton, launches = float(x[0].item()), int(x[1].item())
     F = credited_step_flops(cfg, args.config)
     executed = stats_flops(cfg) + apply_flops(cfg) + newton / interval
+
+    # end to end with host buffers, every rank alike: its gradients come in
+    # from pinned host memory as one flat buffer, the sharded step runs
+    # (reduce-scatter, owner step, all-gather), and the updated weights go
+    # back out from a device snapshot; roots amortised as above
+    e2e = None
+    if not args.no_e2e:
+        shapes_w = [tuple(w.shape) for w in W0]
+        total = sum(int(np.prod(sh)) for sh in shapes_w)
+        pin_g = []
+        for gs in host_grads[:2]:
+            flat = torch.empty(total, dtype=gdt).pin_memory()
+            for v, g in zip(flat_views(flat, shapes_w), gs):
+                v.copy_(torch.from_numpy(g).to(gdt))
+            pin_g.append(flat)
+        pin_w = [torch.empty(total, dtype=torch.float32).pin_memory() for _ in range(2)]
+        dG_flat = [torch.empty(total, dtype=gdt, device=dev) for _ in range(2)]
+        dG = [flat_views(f, shapes_w) for f in dG_flat]
+        snap_flat = [torch.empty(total, dtype=torch.float32, device=dev) for _ in range(2)]
+        snap = [flat_views(f, shapes_w) for f in snap_flat]
+        K = args.steps
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        up_done = [torch.cuda.Event() for _ in range(K)]
+        used = [torch.cuda.Event() for _ in range(K)]
+        snapped = [torch.cuda.Event() for _ in range(K)]
+        down_done = [torch.cuda.Event() for _ in range(K)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        t0.record(stream)
+
+        def upload(j):
+            up.wait_event(t0)
+            if j >= 2:
+                up.wait_event(used[j - 2])
+            with torch.cuda.stream(up):
+                dG_flat[j % 2].copy_(pin_g[j % 2], non_blocking=True)
+            up_done[j].record(up)
+
+        upload(0)
+        for j in range(K):
+            if j + 1 < K:
+                upload(j + 1)
+            stream.wait_event(up_done[j])
+            with torch.cuda.stream(stream):
+                opt.step(W, dG[j % 2], cfg["lr"], False)
+                used[j].record(stream)
+                if j >= 2:
+                    stream.wait_event(down_done[j - 2])
+                for d, w in zip(snap[j % 2], W):
+                    d.copy_(w, non_blocking=True)
+                snapped[j].record(stream)
+            down.wait_event(snapped[j])
+            with torch.cuda.stream(down):
+                pin_w[j % 2].copy_(snap_flat[j % 2], non_blocking=True)
+            down_done[j].record(down)
+        stream.wait_event(down_done[K - 1])
+        t1.record(stream)
+        stream.synchronize()
+        e2e_rank = t0.elapsed_time(t1) / K + max(t_r - t_n, 0.0) / interval
+        e2e_ms = max_over_ranks(e2e_rank, dist if world > 1 else None, dev)
+        h2d = pin_g[0].numel() * pin_g[0].element_size()
+        e2e = {"value": F / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": total * 4 * world,
+               "copies": "every rank: pinned host, its gradients up as one flat buffer and the full "
+                         "updated weights down from a device snapshot, per step, on two copy streams",
+               "amortisation": "K-step loop with host copies, plus (t_root_step - t_step) / root_interval"}
+        del pin_g, pin_w, dG, dG_flat, snap, snap_flat
+
+    # the roofline of rank 0's owned share (its own kernels and work model)
+    roof, every = None, {}
+    if rank == 0 and opt.local is not None:
+        try:
+            peaks, _ = measured_peaks()
+            fp64_peak = fp64_peak_tflops(torch, dev)
+            _, roof, every = roofline(sub, prof, iters, args.steps, len(root_steps), peaks, fp64_peak,
+                                      args.slices, None)
+            if roof is not None:
+                roof["scope"] = "rank 0's owned parameters"
+        except Exception as exc:   # a figure for the line, not a reason to stop the ranks
+            roof = {"error": repr(exc)[:200]}
     if rank == 0:
         line = {"metric": METRIC, "value": F / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -728,7 +810,7 @@ def shard_bench(args, cfg, rank, world, local):
                 "t_step_ms": t_n, "t_root_step_ms": t_r, "timed_region_ms": total_ms,
                 "executed_tflops": executed / (ms * 1e-3) / 1e12,
                 "gpu_launches": launches, "clocks": clk,
-                "cpu_baseline": None, "e2e": None, "roofline": None}
+                "cpu_baseline": None, "e2e": e2e, "roofline": roof, "kernel_roofs": every}
         print(json.dumps(line), flush=True)
     opt.close()
     if world > 1:
