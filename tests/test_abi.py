@@ -167,3 +167,22 @@ def test_binding_signatures_match_the_header():
         assert len(types) == len(args), (name, types, args)
         for t, a in zip(types, args):
             assert _matches(t, a), (name, t, a)
+
+
+def test_binding_checks_tensors_against_the_shapes():
+    """The per-call checks of the Python binding (sizes from the shapes given
+    at construction, contiguity, device) refuse a wrong list before anything
+    reaches the library; built without a context, as the checks need none."""
+    import torch
+    from shampoo_second_order_b200.optimizer import Shampoo
+    opt = object.__new__(Shampoo)
+    opt.shapes = [(4, 3), (5,)]
+    opt._numel = [12, 5]
+    with pytest.raises(ValueError, match="expected 2"):
+        opt._check_tensors([torch.zeros(4, 3)], "grads")
+    with pytest.raises(ValueError, match="contiguous CUDA"):
+        opt._check_tensors([torch.zeros(4, 3), torch.zeros(6)], "grads")          # wrong size
+    with pytest.raises(ValueError, match="contiguous CUDA"):
+        opt._check_tensors([torch.zeros(3, 4).t(), torch.zeros(5)], "grads")      # not contiguous
+    with pytest.raises(ValueError, match="contiguous CUDA"):
+        opt._check_tensors([torch.zeros(4, 3), torch.zeros(5)], "grads")          # host tensors
