@@ -327,7 +327,10 @@ void shampoo_destroy(shampoo_ctx* ctx);
  * n' = n rounded up to 64, at most 2 GiB) in stream order on `stream` from a
  * memory pool the library keeps per device, and frees it back to that pool
  * before returning: the pool keeps the memory (it is not returned to the
- * driver), so calls after the first allocate without the driver.
+ * driver), so calls after the first allocate without the driver.  The
+ * three pinned host ints and two events it polls the iteration with are made
+ * on a host thread's first call on a device and kept for that thread's later
+ * calls there (made again if a device reset released them).
  * Synchronises while it runs, like shampoo_compute_roots.  Returns
  * SHAMPOO_ENOTCONVERGED if any matrix gave up.
  */
